@@ -1,0 +1,137 @@
+"""Seeded synthetic inputs and workload shapes, shared by tests and the bench.
+
+This module holds no arithmetic of the attention method: it only draws random
+numbers and names the workload shapes. Both the CUDA path and the oracle are
+fed from it; neither imports the other.
+
+Generator: counter-based splitmix64 (Steele, Lea, Flood, "Fast splittable
+pseudorandom number generators", OOPSLA 2014): draw i of a stream with seed s is
+mix(s + (i + 1) * 0x9E3779B97F4A7C15). Two 53-bit uniforms per element feed
+the Box-Muller transform, n = sqrt(-2 ln(1 - u1)) * cos(2 pi u2). Values are
+drawn in float64, rounded to float32, then to bfloat16 (round to nearest even).
+Element order is the C order of the requested shape, so a tensor is a pure
+function of (seed, shape) and can be re-drawn anywhere.
+"""
+
+import hashlib
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+_GAMMA = np.uint64(0x9E3779B97F4A7C15)
+_M1 = np.uint64(0xBF58476D1CE4E5B9)
+_M2 = np.uint64(0x94D049BB133111EB)
+_BLOCK = 1 << 22
+
+
+def _mix(z):
+    z = z ^ (z >> np.uint64(30))
+    z = z * _M1
+    z = z ^ (z >> np.uint64(27))
+    z = z * _M2
+    return z ^ (z >> np.uint64(31))
+
+
+def uniforms(seed, start, count):
+    """Draws start..start+count-1 of stream ``seed`` as float64 in [0, 1)."""
+    idx = np.arange(start + 1, start + count + 1, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        z = _mix(np.uint64(seed) + idx * _GAMMA)
+    return (z >> np.uint64(11)).astype(np.float64) * (1.0 / (1 << 53))
+
+
+def normals(seed, count):
+    """``count`` standard normal float64 values of stream ``seed``."""
+    out = np.empty(count, dtype=np.float64)
+    for s in range(0, count, _BLOCK):
+        n = min(_BLOCK, count - s)
+        u = uniforms(seed, 2 * s, 2 * n)
+        out[s:s + n] = np.sqrt(-2.0 * np.log1p(-u[0::2])) * np.cos(2.0 * np.pi * u[1::2])
+    return out
+
+
+def seed_of(*fields):
+    """Stable 64-bit seed of a tuple of names and numbers."""
+    key = "|".join(str(f) for f in fields).encode()
+    return int.from_bytes(hashlib.blake2b(key, digest_size=8).digest(), "little")
+
+
+def normal_bf16(seed, shape, scale=1.0, outlier_frac=0.0, outlier_mag=8.0):
+    """bf16 CPU tensor of N(0, scale^2) values; optionally a Bernoulli
+    ``outlier_frac`` share of elements replaced by +-``outlier_mag``."""
+    count = int(np.prod(shape))
+    vals = normals(seed, count) * scale
+    if outlier_frac > 0.0:
+        pick = uniforms(seed_of(seed, "outlier"), 0, count) < outlier_frac
+        sign = np.where(uniforms(seed_of(seed, "sign"), 0, count) < 0.5, -1.0, 1.0)
+        vals = np.where(pick, sign * outlier_mag, vals)
+    t = torch.from_numpy(vals.astype(np.float32).reshape(shape))
+    return t.to(torch.bfloat16)
+
+
+@dataclass(frozen=True)
+class Workload:
+    """Shape of one synthetic workload (all tensors [B, L, H, D] bf16)."""
+
+    name: str
+    batch: int
+    heads: int
+    head_dim: int
+    frames: int
+    tok_h: int
+    tok_w: int
+    sink: int
+    window: int          # counts the chunk being generated
+    steps: int           # denoising steps per chunk; the last reads the clean tier
+    stream: int          # chunks in the stream used for parity / eviction runs
+    layers: int = 1
+    k_scale: float = 1.0
+    outlier_frac: float = 0.0
+    outlier_mag: float = 8.0
+    notes: str = field(default="", compare=False)
+
+    @property
+    def chunk_len(self):
+        return self.frames * self.tok_h * self.tok_w
+
+    @property
+    def kv_len(self):
+        return (self.sink + self.window) * self.chunk_len
+
+    def shape(self):
+        return (self.batch, self.chunk_len, self.heads, self.head_dim)
+
+    def tensor(self, name, chunk, step=0, layer=0):
+        """Seeded tensor ``name`` of one chunk / step / layer.
+
+        Names: Q, Kc, Vc (current chunk at a denoising step), Kn, Vn (noisy
+        tier copy appended after the chunk), Kcl, Vcl (clean tier copy).
+        """
+        scale = self.k_scale if name.startswith("K") else 1.0
+        return normal_bf16(seed_of(self.name, layer, chunk, step, name), self.shape(),
+                           scale=scale, outlier_frac=self.outlier_frac,
+                           outlier_mag=self.outlier_mag)
+
+    def config_dict(self):
+        return dict(batch=self.batch, heads=self.heads, head_dim=self.head_dim,
+                    frames_per_chunk=self.frames, tok_h=self.tok_h, tok_w=self.tok_w,
+                    sink_chunks=self.sink, window_chunks=self.window)
+
+
+WORKLOADS = {
+    w.name: w
+    for w in (
+        Workload("tiny", 1, 2, 64, 3, 8, 8, sink=1, window=2, steps=2, stream=6,
+                 notes="oracle-sized case"),
+        Workload("s1_540p", 1, 12, 128, 3, 34, 60, sink=1, window=3, steps=4, stream=6,
+                 notes="540p latent chunk, 6120 tokens"),
+        Workload("refiner_720p", 1, 12, 128, 3, 45, 80, sink=1, window=3, steps=1, stream=6,
+                 notes="720p refiner, single clean-tier step"),
+        Workload("backbone_540p_large", 1, 40, 128, 3, 34, 60, sink=1, window=3, steps=4,
+                 stream=32, layers=40, k_scale=0.5, notes="40 layers per step"),
+        Workload("long_stream_stress", 4, 24, 128, 3, 45, 80, sink=2, window=4, steps=4,
+                 stream=200, outlier_frac=0.01, outlier_mag=8.0,
+                 notes="3 noisy steps + 1 clean step per chunk, 1% outliers of +-8"),
+    )
+}
