@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of one chunk-step of block-causal sink + window TwinCache attention.
+
+A step is one chunk of the stream at steady state (window full, eviction on):
+every denoising step's attention (sa_stage_keys + sa_attend_staged; the last
+step reads the clean tier) followed by the append of the chunk's noisy and
+clean K/V (sa_append_chunk x2). Inputs are seeded synthetic bf16 tensors of the
+workload's shape, resident in HBM before the timed region.
+
+Prints ONE JSON line (rank 0). ``value`` is attention TFLOP/s over all ranks
+(FLOPs = 4 * B * H * L * Lkv * D per attention); ``ms_per_step`` the time of a
+chunk-step. With torchrun each rank runs its own independent stream (weak
+scaling, no data-path collective); the barrier and the max over ranks of the
+device time use NCCL.
+
+``--impl reference`` times the float64 CPU oracle on the host cores on a
+bounded sample of the same workload instead.
+"""
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms per chunk-step and attention TFLOP/s (% of B200 bf16 peak) at 720p shape"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 2 ** 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="refiner_720p")
+    ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def attend_flops(w):
+    return 4.0 * w.batch * w.heads * w.chunk_len * w.kv_len * w.head_dim
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_traffic(kernel_file, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the kernel source as it is now; else None."""
+    src = os.path.join(ROOT, "block_causal_streaming_sa_b200", "csrc", "kernels", kernel_file)
+    summ = os.path.join(ROOT, "profiles", f"attend_tc_{workload}.md")
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        text = open(summ).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*(\d+)\s*;\s*source_sha256_16:\s*([0-9a-f]+)", text)
+    if m and m.group(2) == sha:
+        return int(m.group(1))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, bus_id):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", bus_id],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, power, reasons = [], [], [], set()
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "power_w_median": statistics.median(power), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def bus_id_of(dev):
+    import torch
+
+    p = torch.cuda.get_device_properties(dev)
+    return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+# ------------------------------------------------------------------ oracle (CPU) legs
+
+
+class OracleSample:
+    """The float64 oracle on a bounded sample of the workload: the generating
+    chunk at steady state, one (batch, head) pair and a few query rows per call."""
+
+    def __init__(self, w):
+        import numpy as np
+        import torch
+
+        from oracle.stream import CLEAN, NOISY, OracleConfig, StreamOracle
+
+        self.np = np
+        self.w = w
+        cfg = OracleConfig(w.batch, w.heads, w.head_dim, w.frames, w.tok_h, w.tok_w, w.sink,
+                           w.window)
+        self.orc = StreamOracle(cfg)
+        f64 = lambda t: t.to(torch.float64).numpy()  # noqa: E731
+        pool = [{n: f64(w.tensor(n, c)) for n in ("Kn", "Vn", "Kcl", "Vcl")} for c in range(2)]
+        for c in range(w.sink + w.window - 1):
+            s = pool[c % 2]
+            self.orc.append(NOISY, s["Kn"], s["Vn"])
+            self.orc.append(CLEAN, s["Kcl"], s["Vcl"])
+        self.cur = {n: f64(w.tensor(n, 9)) for n in ("Q", "Kc", "Vc")}
+        self.rng = np.random.default_rng(3)
+        self.calls = 0
+
+    def run(self, rows):
+        """One sample: `rows` query rows of one (b, h); returns its FLOPs."""
+        w = self.w
+        bh = self.calls % (w.batch * w.heads)
+        self.calls += 1
+        b, h = divmod(bh, w.heads)
+        sel = self.rng.choice(w.chunk_len, size=rows, replace=False)
+        self.orc.attend(self.cur["Q"], self.cur["Kc"], self.cur["Vc"], True, rows=sel,
+                        heads=[h], batches=[b])
+        return 4.0 * rows * w.kv_len * w.head_dim
+
+    def calibrate(self, seconds):
+        """Rows per call such that one call takes about `seconds`."""
+        t = time.perf_counter()
+        self.run(16)
+        t16 = time.perf_counter() - t
+        t = time.perf_counter()
+        self.run(128)
+        t128 = time.perf_counter() - t
+        per_row = max((t128 - t16) / 112, 1e-6)
+        fixed = max(t16 - 16 * per_row, 0.0)
+        return int(min(self.w.chunk_len, max(16, (seconds - fixed) / per_row)))
+
+
+def cpu_baseline(w, seconds):
+    o = OracleSample(w)
+    rows = o.calibrate(min(seconds / 3, 5.0))
+    flops, t0 = 0.0, time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        flops += o.run(rows)
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{o.calls - 2} calls x {rows} query rows of one (b,h) each, "
+                      f"all {w.kv_len} keys, final (clean-tier) step at steady state, "
+                      f"{dt:.1f} s of float64 numpy on the host"}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    o = OracleSample(w)
+    rows = o.calibrate(0.15)
+    for _ in range(args.warmup):
+        o.run(rows)
+    flops, t0 = 0.0, time.perf_counter()
+    for _ in range(args.steps):
+        flops += o.run(rows)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    sample = (f"each step: {rows} query rows of one (b,h) over all {w.kv_len} keys "
+              f"(float64 numpy oracle, host cores)")
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": w.name, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU leg
+
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import block_causal_streaming_sa_b200 as sa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    stream = torch.cuda.Stream(device=dev)
+    names = ("Q", "Kc", "Vc", "Kn", "Vn", "Kcl", "Vcl")
+    pool_host = [{n: w.tensor(n, 100 + c, layer=rank).pin_memory() for n in names}
+                 for c in range(2)]
+    pool = [{n: t.to(dev) for n, t in s.items()} for s in pool_host]
+    out = torch.empty(w.shape(), dtype=torch.bfloat16, device=dev)
+    out_host = torch.empty(w.shape(), dtype=torch.bfloat16).pin_memory()
+
+    attn = sa.StreamingAttention(w.config_dict(), device=dev)
+    h = attn.handle
+    sp = stream.cuda_stream
+    flops = attend_flops(w)
+    steps_per_chunk = w.steps
+    appends_per_chunk = 2
+
+    def chunk_step(s, ev=None):
+        """One chunk: every denoising step's attention, then the two appends."""
+        for k in range(steps_per_chunk):
+            final = k == steps_per_chunk - 1
+            sa.sa_stage_keys(h, s["Kc"].data_ptr(), sp)
+            if ev is not None:
+                ev[0][k].record(stream)
+            sa.sa_attend_staged(h, s["Q"].data_ptr(), s["Vc"].data_ptr(), final, out.data_ptr(),
+                                0, sp)
+            if ev is not None:
+                ev[1][k].record(stream)
+        if ev is not None:
+            ev[2].record(stream)
+        sa.sa_append_chunk(h, sa.SA_TIER_NOISY, s["Kn"].data_ptr(), s["Vn"].data_ptr(), sp)
+        sa.sa_append_chunk(h, sa.SA_TIER_CLEAN, s["Kcl"].data_ptr(), s["Vcl"].data_ptr(), sp)
+        if ev is not None:
+            ev[3].record(stream)
+
+    with torch.cuda.stream(stream):
+        # Fill the window so every timed chunk attends to S + W chunks.
+        for c in range(w.sink + w.window - 1):
+            s = pool[c % 2]
+            sa.sa_append_chunk(h, sa.SA_TIER_NOISY, s["Kn"].data_ptr(), s["Vn"].data_ptr(), sp)
+            sa.sa_append_chunk(h, sa.SA_TIER_CLEAN, s["Kcl"].data_ptr(), s["Vcl"].data_ptr(), sp)
+        for i in range(args.warmup):
+            chunk_step(pool[i % 2])
+        stream.synchronize()
+
+        mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+        evs = [([mk() for _ in range(steps_per_chunk)], [mk() for _ in range(steps_per_chunk)],
+                mk(), mk()) for _ in range(args.steps)]
+        start, stop = mk(), mk()
+        barrier()
+        torch.cuda.synchronize(dev)
+        clocks = ClockSampler(bus_id_of(dev)) if rank == 0 else None
+        start.record(stream)
+        for i in range(args.steps):
+            chunk_step(pool[i % 2], evs[i])
+        stop.record(stream)
+        stream.synchronize()
+        torch.cuda.synchronize(dev)
+        clock_info = clocks.stop() if clocks is not None else None
+        barrier()
+        ms_local = start.elapsed_time(stop)
+        attend_ms = [e[0][k].elapsed_time(e[1][k]) for e in evs for k in range(steps_per_chunk)]
+        append_ms = [e[2].elapsed_time(e[3]) for e in evs]
+        assert attn.status(stream) == sa.SA_OK, "device status word reports a timeout"
+
+        # End to end through the public API with host buffers: H2D of the step's
+        # seven input tensors, the chunk-step, D2H of the output.
+        e2e_steps = max(1, args.e2e_steps)
+        h2d = sum(t.numel() * t.element_size() for t in pool_host[0].values())
+        d2h = out_host.numel() * out_host.element_size()
+        dev_bufs = {n: torch.empty_like(t) for n, t in pool[0].items()}
+        for i in range(2):
+            for n, t in pool_host[i % 2].items():
+                dev_bufs[n].copy_(t, non_blocking=True)
+            chunk_step(dev_bufs)
+            out_host.copy_(out, non_blocking=True)
+        stream.synchronize()
+        barrier()
+        e0, e1 = mk(), mk()
+        e0.record(stream)
+        for i in range(e2e_steps):
+            for n, t in pool_host[i % 2].items():
+                dev_bufs[n].copy_(t, non_blocking=True)
+            chunk_step(dev_bufs)
+            out_host.copy_(out, non_blocking=True)
+        e1.record(stream)
+        stream.synchronize()
+        e2e_ms_local = e0.elapsed_time(e1)
+        barrier()
+
+    ms_max = max_over_ranks(ms_local)
+    e2e_ms_max = max_over_ranks(e2e_ms_local)
+    total_flops = flops * steps_per_chunk * args.steps * world
+    value = total_flops / (ms_max * 1e-3) / 1e12
+    e2e_value = flops * steps_per_chunk * e2e_steps * world / (e2e_ms_max * 1e-3) / 1e12
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_seconds)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    attend_avg = statistics.fmean(attend_ms)
+    achieved = flops / (attend_avg * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    append_bytes = appends_per_chunk * 2 * 2 * (w.batch * w.chunk_len * w.heads * w.head_dim * 2)
+    append_gbs = append_bytes / (statistics.fmean(append_ms) * 1e-3) / 1e9
+    cache_bytes_read = 2 * (w.kv_len - w.chunk_len) * w.batch * w.heads * w.head_dim * 2
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
+            "chunk_tokens": w.chunk_len, "kv_tokens": w.kv_len, "sink_chunks": w.sink,
+            "window_chunks": w.window, "denoise_steps_per_chunk": w.steps,
+            "step": "all denoising attentions of one chunk + noisy and clean append",
+            "l2": f"inputs larger than L2: {cache_bytes_read / 2**20:.0f} MiB of cached K/V "
+                  f"read per attention vs {L2_BYTES / 2**20:.0f} MiB L2",
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+        },
+        "roofline": {
+            "bound": "tensor", "kernel": "attend_tc_kernel<128>",
+            "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "peak_kind": f"bf16 sustained ({peak_src})", "frac_of_burst_peak": achieved / burst,
+            "traffic": kernel_traffic("attend_tc.cuh", w.name),
+            "flops_per_launch": flops, "avg_launch_ms": attend_avg,
+        },
+        "append": {"ms": statistics.fmean(append_ms), "GB_per_s": append_gbs,
+                   "frac_of_hbm": append_gbs / float(peaks.get("hbm_gbs", 6650.0))},
+        "ms_per_attention": attend_avg,
+        "attention_tflops_kernel": achieved,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms_max / e2e_steps},
+        "gpu_launches": args.steps * (2 * steps_per_chunk + appends_per_chunk),
+        "clocks": clock_info,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    from sa_inputs import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,16 @@
+"""Block-causal sink + window TwinCache attention for B200 (sm_100a).
+
+The compute lives in ``libsa.so`` (CUDA kernels behind a C ABI, include/sa.h).
+``_binding`` exposes each C entry point under its own name; ``StreamingAttention``
+is a small convenience wrapper that owns the device buffer (allocated through
+PyTorch) and passes tensors' device pointers and the current CUDA stream.
+"""
+
+from ._binding import (  # noqa: F401
+    SA_OK, SA_ERR_INVALID_ARG, SA_ERR_STATE, SA_ERR_UNSUPPORTED, SA_ERR_CUDA, SA_ERR_TIMEOUT,
+    SA_TIER_NOISY, SA_TIER_CLEAN, SaConfig, SaError, make_config, lib, header_symbols,
+    sa_validate_config, sa_required_bytes, sa_create, sa_destroy, sa_reset, sa_append_chunk,
+    sa_attend, sa_stage_keys, sa_attend_staged, sa_debug_attend_simt, sa_chunk_count, sa_debug_layout, sa_plan, sa_slot_of,
+    sa_get_status, last_error,
+)
+from .stream import StreamingAttention  # noqa: F401

@@ -1,0 +1,189 @@
+"""ctypes binding of libsa.so: one Python function per C entry point, same names.
+
+Argument marshalling only: pointers are plain integers (device addresses, or
+host addresses for the introspection calls), streams are cudaStream_t handles
+as integers. Every compute step runs in the library's CUDA kernels; if the
+library is missing this module raises instead of falling back to anything.
+"""
+
+import ctypes
+import os
+import re
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libsa.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "sa.h")
+
+SA_OK = 0
+SA_ERR_INVALID_ARG = 1
+SA_ERR_STATE = 2
+SA_ERR_UNSUPPORTED = 3
+SA_ERR_CUDA = 4
+SA_ERR_TIMEOUT = 5
+SA_TIER_NOISY = 0
+SA_TIER_CLEAN = 1
+SA_MAX_ATTENDED = 16
+
+
+class SaConfig(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("frames_per_chunk", ctypes.c_int32),
+        ("tok_h", ctypes.c_int32),
+        ("tok_w", ctypes.c_int32),
+        ("sink_chunks", ctypes.c_int32),
+        ("window_chunks", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_float),
+        ("rope_theta", ctypes.c_float),
+    ]
+
+
+class SaError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"{status_name(status)}: {message}")
+        self.status = status
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I32P = ctypes.POINTER(ctypes.c_int32)
+_CFGP = ctypes.POINTER(SaConfig)
+
+_SIGNATURES = {
+    "sa_validate_config": (_I, [_CFGP]),
+    "sa_required_bytes": (ctypes.c_size_t, [_CFGP]),
+    "sa_create": (_I, [_CFGP, _P, ctypes.c_size_t, ctypes.POINTER(_P)]),
+    "sa_destroy": (_I, [_P]),
+    "sa_reset": (_I, [_P]),
+    "sa_append_chunk": (_I, [_P, _I, _P, _P, _P]),
+    "sa_attend": (_I, [_P, _P, _P, _P, _I, _P, _P, _P]),
+    "sa_stage_keys": (_I, [_P, _P, _P]),
+    "sa_attend_staged": (_I, [_P, _P, _P, _I, _P, _P, _P]),
+    "sa_debug_attend_simt": (_I, [_P, _P, _P, _P, _I, _P, _P, _P]),
+    "sa_chunk_count": (_I, [_P, _I]),
+    "sa_debug_layout": (_I, [_P, _I, _I32P, _I]),
+    "sa_plan": (_I, [_CFGP, ctypes.c_int32, _I32P, _I32P, _I32P, _I]),
+    "sa_slot_of": (_I, [_CFGP, ctypes.c_int32]),
+    "sa_get_status": (_I, [_P, _P]),
+    "sa_last_error": (ctypes.c_char_p, [_P]),
+    "sa_status_string": (ctypes.c_char_p, [_I]),
+}
+
+
+def lib():
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m block_causal_streaming_sa_b200.build` (there is no fallback)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = handle
+    return _lib
+
+
+def header_symbols():
+    """Entry points declared in include/sa.h."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SA_API\s+[\w\s\*]+?\b(sa_\w+)\s*\(", text)))
+
+
+def status_name(status):
+    return lib().sa_status_string(int(status)).decode()
+
+
+def last_error(handle=None):
+    return lib().sa_last_error(handle).decode()
+
+
+def _check(status, handle=None):
+    if status != SA_OK:
+        raise SaError(status, last_error(handle))
+
+
+def make_config(batch, heads, head_dim, frames_per_chunk, tok_h, tok_w, sink_chunks,
+                window_chunks, softmax_scale=0.0, rope_theta=0.0):
+    return SaConfig(batch, heads, head_dim, frames_per_chunk, tok_h, tok_w, sink_chunks,
+                    window_chunks, softmax_scale, rope_theta)
+
+
+def sa_validate_config(cfg):
+    return lib().sa_validate_config(ctypes.byref(cfg))
+
+
+def sa_required_bytes(cfg):
+    return lib().sa_required_bytes(ctypes.byref(cfg))
+
+
+def sa_create(cfg, dev_buf, nbytes):
+    out = _P()
+    _check(lib().sa_create(ctypes.byref(cfg), _P(dev_buf), nbytes, ctypes.byref(out)))
+    return out
+
+
+def sa_destroy(handle):
+    _check(lib().sa_destroy(handle))
+
+
+def sa_reset(handle):
+    _check(lib().sa_reset(handle), handle)
+
+
+def sa_append_chunk(handle, tier, K, V, stream=0):
+    _check(lib().sa_append_chunk(handle, tier, _P(K), _P(V), _P(stream)), handle)
+
+
+def sa_attend(handle, Q, Kc, Vc, step_is_final, O, lse=0, stream=0):
+    _check(lib().sa_attend(handle, _P(Q), _P(Kc), _P(Vc), int(bool(step_is_final)), _P(O),
+                           _P(lse or None), _P(stream)), handle)
+
+
+def sa_stage_keys(handle, Kc, stream=0):
+    _check(lib().sa_stage_keys(handle, _P(Kc), _P(stream)), handle)
+
+
+def sa_attend_staged(handle, Q, Vc, step_is_final, O, lse=0, stream=0):
+    _check(lib().sa_attend_staged(handle, _P(Q), _P(Vc), int(bool(step_is_final)), _P(O),
+                                  _P(lse or None), _P(stream)), handle)
+
+
+def sa_debug_attend_simt(handle, Q, Kc, Vc, step_is_final, O, lse=0, stream=0):
+    _check(lib().sa_debug_attend_simt(handle, _P(Q), _P(Kc), _P(Vc), int(bool(step_is_final)),
+                                      _P(O), _P(lse or None), _P(stream)), handle)
+
+
+def sa_chunk_count(handle, tier):
+    return lib().sa_chunk_count(handle, tier)
+
+
+def sa_debug_layout(handle, tier, n):
+    buf = (ctypes.c_int32 * n)()
+    m = lib().sa_debug_layout(handle, tier, buf, n)
+    if m < 0:
+        raise SaError(-m, last_error(handle))
+    return list(buf[:m])
+
+
+def sa_plan(cfg, chunk):
+    """(ids, slots, t_base) of chunk `chunk`'s attention, computed by the library."""
+    cap = SA_MAX_ATTENDED
+    ids, slots, tb = ((ctypes.c_int32 * cap)() for _ in range(3))
+    n = lib().sa_plan(ctypes.byref(cfg), chunk, ids, slots, tb, cap)
+    if n < 0:
+        raise SaError(-n, last_error())
+    return list(ids[:n]), list(slots[:n]), list(tb[:n])
+
+
+def sa_slot_of(cfg, chunk):
+    return lib().sa_slot_of(ctypes.byref(cfg), chunk)
+
+
+def sa_get_status(handle, stream=0):
+    return lib().sa_get_status(handle, _P(stream))

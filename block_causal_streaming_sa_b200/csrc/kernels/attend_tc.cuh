@@ -1,0 +1,455 @@
+// Tensor-core attention of one chunk over its sink + window chunks (sm_100a).
+//
+// What it computes ("Vidu S2 vs PixVerse R2：实时视频的两条技术路线", sections
+// 「实时」改变了什么 and 选择三：有上限的记忆): for every query row of the chunk
+// being generated, softmax attention over the keys of the cached sink and window
+// chunks of one TwinCache tier plus the chunk's own keys, with the temporal RoPE
+// position of chunk j relocated to rank(j) * F.
+//
+// Design (B200):
+//  * persistent CTAs, one per SM; a work tile is two 128-row query tiles of one
+//    (batch, head), so every K/V tile brought in by TMA feeds two MMAs;
+//  * warp 0 (one lane): TMA producer over a ring of NSTAGE 128x D bf16 tiles,
+//    K_0 V_0 K_1 V_1 ..., 128-byte swizzle, straight from the cache slots and
+//    from the caller's V (no gather copy);
+//  * warp 1 (one lane): tcgen05.mma issuer. S_i = Q_i K^T (SS form, both
+//    operands K-major in shared memory) into TMEM, then O_i += P_i V (TS form:
+//    P_i read from TMEM, written over the upper half of S_i, V MN-major in shared memory);
+//    the two query tiles ping-pong so one tile's softmax overlaps the other's
+//    MMAs;
+//  * warps 2-5 / 6-9: one warpgroup per query tile, thread = query row =
+//    TMEM lane. Each writes its rotated query tile into shared memory, runs the
+//    online softmax on S rows read from TMEM (no cross-thread reduction: a
+//    thread owns a whole row), writes P back as bf16, rescales O in TMEM only
+//    when the running max grows by more than 2^8, and runs the epilogue;
+//  * RoPE: keys are stored rotated by their in-chunk position; the relocated
+//    temporal base rank(j) * F of the attended chunk is applied by re-turning
+//    the temporal band of the query tile when the key stream moves to the next
+//    chunk, before the first QK^T MMA of that chunk.
+// All mbarrier waits are bounded (see ptx.cuh); on a timeout every role drains
+// its outstanding async work, TMEM is freed and the device status word is set.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "../sa_internal.h"
+#include "ptx.cuh"
+#include "rope.cuh"
+
+namespace sa {
+
+template <int D>
+struct TcShape {
+  static constexpr int BM = 128;                 // query rows per tile (= TMEM lanes)
+  static constexpr int BN = 128;                 // keys per K/V tile
+  static constexpr int KBLK = D / 64;            // 64-element (128-byte) swizzle atoms per row
+  static constexpr int kTile = BM * D * 2;       // bytes of a Q, K or V tile (BM == BN)
+  static constexpr int kBox = BN * 128;          // bytes of one 64-column TMA box
+  static constexpr int NSTAGE = (D == 128) ? 4 : 8;
+  static constexpr int kThreads = 320;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = 2 * kTile;
+  static constexpr int kOffQRaw = kOffKV + NSTAGE * kTile;  // raw temporal chunks of both Q tiles
+  static constexpr int kQRawRow = ((D - 4 * (D / 6) + 7) / 8) * 16;
+  static constexpr int kOffBar = kOffQRaw + 2 * BM * kQRawRow;
+  static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + barrier area + alignment slack
+  static constexpr int kTmemCols = 512;
+  static constexpr int kDt = D - 4 * (D / 6);             // temporal band width
+  static constexpr int kTChunks = (kDt + 7) / 8;           // 16-byte chunks holding it
+  static constexpr uint32_t kIdescQK = ptx::idesc_bf16_f32(BM, BN, 0);
+  static constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(BM, D, 1);
+  __host__ __device__ static constexpr int col_s(int i) { return i * 128; }
+  __host__ __device__ static constexpr int col_o(int i) { return 256 + i * D; }
+  __host__ __device__ static constexpr int col_p(int i) { return i * 128 + 64; }  // bf16 P
+  // barrier indices
+  __host__ __device__ static constexpr int FULL(int s) { return s; }
+  __host__ __device__ static constexpr int EMPTY(int s) { return NSTAGE + s; }
+  __host__ __device__ static constexpr int QREADY(int i) { return 2 * NSTAGE + i; }
+  __host__ __device__ static constexpr int SFULL(int i) { return 2 * NSTAGE + 2 + i; }
+  __host__ __device__ static constexpr int PFULL(int i) { return 2 * NSTAGE + 4 + i; }
+  __host__ __device__ static constexpr int OFINAL(int i) { return 2 * NSTAGE + 6 + i; }
+  __host__ __device__ static constexpr int DRAIN() { return 2 * NSTAGE + 8; }
+  static constexpr int kNumBars = 2 * NSTAGE + 9;
+  static_assert(kNumBars * 8 <= 224, "barrier area");
+  static_assert(kSmemBytes <= 232448, "shared memory");
+};
+
+// Offset of 16-byte chunk c of row r in a 128-byte-swizzled K-major tile of 128 rows.
+__device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
+  return static_cast<uint32_t>((c >> 3) * (128 * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    attend_tc_kernel(const __grid_constant__ CUtensorMap tm_cache,
+                     const __grid_constant__ CUtensorMap tm_kcur,
+                     const __grid_constant__ CUtensorMap tm_vcur,
+                     const __grid_constant__ AttendParams p) {
+  using T = TcShape<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = ptx::smem_addr(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  const uint32_t sbase = ptx::smem_addr(smem);
+  const uint32_t bar0 = sbase + T::kOffBar;
+  auto bar = [&](int idx) { return bar0 + 8u * static_cast<uint32_t>(idx); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + T::kOffBar + 224);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + T::kOffBar + 228);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < T::NSTAGE; ++s) {
+      ptx::mbar_init(bar(T::FULL(s)), 1);
+      ptx::mbar_init(bar(T::EMPTY(s)), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(bar(T::QREADY(i)), 128);
+      ptx::mbar_init(bar(T::SFULL(i)), 1);
+      ptx::mbar_init(bar(T::PFULL(i)), 128);
+      ptx::mbar_init(bar(T::OFINAL(i)), 1);
+    }
+    ptx::mbar_init(bar(T::DRAIN()), 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_addr(tmem_slot), T::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+
+  const int n_qt = (p.L + T::BM - 1) / T::BM;
+  const int n_pairs = (n_qt + 1) / 2;
+  const int n_work = p.B * p.H * n_pairs;
+  int n_kt_total = 0;
+  for (int g = 0; g < p.n_groups; ++g) n_kt_total += (p.groups[g].len + T::BN - 1) / T::BN;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      ptx::tma_prefetch_desc(&tm_cache);
+      ptx::tma_prefetch_desc(&tm_kcur);
+      ptx::tma_prefetch_desc(&tm_vcur);
+      int stage = 0;
+      uint32_t phase = 0, filled_mask = 0, filled_parity = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x) {
+        const int bh = w / n_pairs;
+        const int b = bh / p.H, h = bh - b * p.H;
+        for (int g = 0; ok && g < p.n_groups; ++g) {
+          const AttendGroup grp = p.groups[g];
+          const int nkt = (grp.len + T::BN - 1) / T::BN;
+          for (int t = 0; ok && t < nkt; ++t) {
+            for (int kv = 0; kv < 2; ++kv) {
+              if (!ptx::mbar_wait(bar(T::EMPTY(stage)), phase ^ 1u, abort_flag, p.status)) {
+                ok = false;
+                break;
+              }
+              const uint32_t full = bar(T::FULL(stage));
+              ptx::mbar_arrive_expect_tx(full, T::kTile);
+              const uint32_t dst = sbase + T::kOffKV + stage * T::kTile;
+              for (int kb = 0; kb < T::KBLK; ++kb) {
+                if (grp.src == 0) {
+                  const int plane = ((grp.slot * 2 + kv) * p.B + b) * p.H + h;
+                  ptx::tma_load_3d(dst + kb * T::kBox, &tm_cache, full, kb * 64, t * T::BN, plane);
+                } else if (kv == 0) {
+                  ptx::tma_load_3d(dst + kb * T::kBox, &tm_kcur, full, kb * 64, t * T::BN,
+                                   b * p.H + h);
+                } else {
+                  ptx::tma_load_4d(dst + kb * T::kBox, &tm_vcur, full, kb * 64, h, t * T::BN, b);
+                }
+              }
+              filled_mask |= 1u << stage;
+              filled_parity = (filled_parity & ~(1u << stage)) | (phase << stage);
+              if (++stage == T::NSTAGE) {
+                stage = 0;
+                phase ^= 1u;
+              }
+            }
+          }
+        }
+      }
+      // Let every issued copy land before the CTA can exit.
+      volatile int no_abort = 0;
+      for (int s = 0; s < T::NSTAGE; ++s)
+        if (filled_mask & (1u << s))
+          ptx::mbar_wait(bar(T::FULL(s)), (filled_parity >> s) & 1u, &no_abort, p.status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t pf_phase[2] = {0u, 0u};
+      bool ok = true;
+      auto take_stage = [&](int& s_out) -> bool {
+        s_out = stage;
+        const bool r = ptx::mbar_wait(bar(T::FULL(stage)), phase, abort_flag, p.status);
+        if (++stage == T::NSTAGE) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        return r;
+      };
+      auto issue_s = [&](int i, int sk) {
+        const uint32_t qa = sbase + T::kOffQ + i * T::kTile;
+        const uint32_t kb = sbase + T::kOffKV + sk * T::kTile;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * T::kBox + (kk & 3) * 32;
+          ptx::umma_ss(tmem + T::col_s(i), ptx::smem_desc_sw128(qa + off, 16, 1024),
+                       ptx::smem_desc_sw128(kb + off, 16, 1024), T::kIdescQK, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int i, int sv, bool accumulate) {
+        const uint32_t vb = sbase + T::kOffKV + sv * T::kTile;
+#pragma unroll
+        for (int kk = 0; kk < T::BN / 16; ++kk) {
+          ptx::umma_ts(tmem + T::col_o(i), tmem + T::col_p(i) + kk * 8,
+                       ptx::smem_desc_sw128(vb + kk * 16 * 128, T::kBox, 1024), T::kIdescPV,
+                       (accumulate || kk > 0) ? 1u : 0u);
+        }
+      };
+      int wi = 0;
+      for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++wi) {
+        int sk = 0, sv = 0;
+        if (!take_stage(sk)) break;
+        ptx::tc_fence_after();
+        for (int i = 0; i < 2; ++i) {
+          if (!ptx::mbar_wait(bar(T::QREADY(i)), wi & 1, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          issue_s(i, sk);
+          ptx::umma_commit(bar(T::SFULL(i)));
+        }
+        if (!ok) break;
+        ptx::umma_commit(bar(T::EMPTY(sk)));
+        for (int kt = 0; ok && kt < n_kt_total; ++kt) {
+          const bool has_next = kt + 1 < n_kt_total;
+          if (!take_stage(sv) || (has_next && !take_stage(sk))) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          for (int i = 0; i < 2; ++i) {
+            if (!ptx::mbar_wait(bar(T::PFULL(i)), pf_phase[i], abort_flag, p.status)) {
+              ok = false;
+              break;
+            }
+            pf_phase[i] ^= 1u;
+            ptx::tc_fence_after();
+            issue_pv(i, sv, kt > 0);
+            if (i == 1) ptx::umma_commit(bar(T::EMPTY(sv)));
+            if (!has_next) ptx::umma_commit(bar(T::OFINAL(i)));
+            if (has_next) {
+              issue_s(i, sk);
+              ptx::umma_commit(bar(T::SFULL(i)));
+            }
+          }
+          if (ok && has_next) ptx::umma_commit(bar(T::EMPTY(sk)));
+        }
+      }
+      // Every MMA issued so far must finish before TMEM is released.
+      volatile int no_abort = 0;
+      ptx::umma_commit(bar(T::DRAIN()));
+      ptx::mbar_wait(bar(T::DRAIN()), 0, &no_abort, p.status);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int i = (warp - 2) >> 2;  // query tile of this warpgroup
+    const int quarter = warp & 3;   // TMEM lane quarter this warp may access
+    const int r = quarter * 32 + lane;
+    const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + t_lane + T::col_s(i);
+    const uint32_t tO = tmem + t_lane + T::col_o(i);
+    const uint32_t q_smem = sbase + T::kOffQ + i * T::kTile;
+    uint32_t s_phase = 0;
+    bool ok = true;
+    int wi = 0;
+    for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++wi) {
+      const int bh = w / n_pairs, pair = w - bh * n_pairs;
+      const int b = bh / p.H, h = bh - b * p.H;
+      const int q_row = (2 * pair + i) * T::BM + r;
+      const bool valid = q_row < p.L;
+      const int qr = valid ? q_row : 0;
+      const int f = qr / p.rope.frame_tokens;
+      const int y = (qr / p.rope.tok_w) % p.rope.tok_h;
+      const int x = qr % p.rope.tok_w;
+      const size_t row_off = ((static_cast<size_t>(b) * p.L + qr) * p.H + h) * D;
+
+      // Rotated query tile for the first attended chunk; the raw temporal chunks
+      // are kept in shared memory for the re-turns at chunk switches.
+      const uint32_t q_raw = sbase + T::kOffQRaw + (i * T::BM + r) * T::kQRawRow;
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(p.q + row_off);
+        const int td0 = p.groups[0].t_delta;
+#pragma unroll 2
+        for (int c = 0; c < D / 8; ++c) {
+          uint4 v = valid ? ld_nc_v4(src + c) : make_uint4(0u, 0u, 0u, 0u);
+          if (c < T::kTChunks) st_shared_v4(q_raw + c * 16, v);
+          st_shared_v4(q_smem + sw128_offset(r, c), rope_chunk(v, c, p.rope, td0 + f, y, x));
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(bar(T::QREADY(i)));
+      }
+
+      float m = -INFINITY, lsum = 0.f;
+      int kt = 0;
+      for (int g = 0; ok && g < p.n_groups; ++g) {
+        const int len = p.groups[g].len;
+        const int nkt = (len + T::BN - 1) / T::BN;
+        for (int t = 0; t < nkt; ++t, ++kt) {
+          if (!ptx::mbar_wait(bar(T::SFULL(i)), s_phase, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          s_phase ^= 1u;
+          ptx::tc_fence_after();
+          // Scores of keys [col0, col0 + 64) of this row, keys past the chunk end masked.
+          const int nvalid = min(T::BN, len - t * T::BN);
+          uint32_t sr[2][32];
+          auto load_half = [&](int col0) {
+            ptx::tmem_ld32(tS + col0, sr[0]);
+            ptx::tmem_ld32(tS + col0 + 32, sr[1]);
+            ptx::tmem_wait_ld();
+            if (nvalid < col0 + 64) {
+#pragma unroll
+              for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                  if (col0 + j * 32 + c >= nvalid) sr[j][c] = __float_as_uint(-INFINITY);
+            }
+          };
+          auto half_max = [&]() {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+              for (int c = 0; c < 32; ++c) mx = fmaxf(mx, __uint_as_float(sr[j][c]));
+            return mx;
+          };
+          load_half(0);
+          float mx = half_max();
+          load_half(64);
+          mx = fmaxf(mx, half_max());
+          const float m_new = fmaxf(m, mx * p.scale_log2);
+          const bool need = m_new > m + 8.0f;
+          float alpha = 1.f;
+          if (need) {
+            alpha = ptx::ex2(m - m_new);
+            m = m_new;
+          }
+          // P = 2^(s * scale * log2 e - m) as bf16 pairs in columns 64..127 of the S
+          // region (P of key k in column 64 + k / 2). Keys 64..127 first, from the
+          // registers: their P overwrites scores of keys 96..127, already read. Then
+          // keys 0..63 after reloading them: their P overwrites keys 64..95, also read.
+          float rs = 0.f;
+          auto exp_store = [&](int pcol) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int c = 0; c < 16; ++c) {
+                const float p0 =
+                    ptx::ex2(fmaf(__uint_as_float(sr[j][2 * c]), p.scale_log2, -m));
+                const float p1 =
+                    ptx::ex2(fmaf(__uint_as_float(sr[j][2 * c + 1]), p.scale_log2, -m));
+                rs += p0 + p1;
+                pk[c] = ptx::pack_bf16x2(p0, p1);
+              }
+              ptx::tmem_st16(tS + pcol + j * 16, pk);
+            }
+          };
+          exp_store(96);
+          load_half(0);
+          exp_store(64);
+          lsum = lsum * alpha + rs;
+          if (__any_sync(0xffffffffu, need && kt > 0)) {
+#pragma unroll
+            for (int j = 0; j < D / 32; ++j) {
+              uint32_t o[32];
+              ptx::tmem_ld32(tO + j * 32, o);
+              ptx::tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+              ptx::tmem_st32(tO + j * 32, o);
+            }
+          }
+          if (t == nkt - 1 && g + 1 < p.n_groups) {
+            const int td = p.groups[g + 1].t_delta;
+#pragma unroll 2
+            for (int c = 0; c < T::kTChunks; ++c)
+              st_shared_v4(q_smem + sw128_offset(r, c),
+                           rope_chunk(ld_shared_v4(q_raw + c * 16), c, p.rope, td + f, y, x));
+            ptx::fence_proxy_async_smem();
+          }
+          ptx::tmem_wait_st();
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(bar(T::PFULL(i)));
+        }
+      }
+      if (!ok) break;
+
+      // Epilogue: O / l -> bf16 rows of [B, L, H, D]; optional natural-log LSE.
+      if (!ptx::mbar_wait(bar(T::OFINAL(i)), wi & 1, abort_flag, p.status)) break;
+      ptx::tc_fence_after();
+      const float inv = 1.f / lsum;
+      uint4* dst = reinterpret_cast<uint4*>(p.o + row_off);
+#pragma unroll 1
+      for (int j = 0; j < D / 32; ++j) {
+        uint32_t o[32];
+        ptx::tmem_ld32(tO + j * 32, o);
+        ptx::tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 u;
+            u.x = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv,
+                                   __uint_as_float(o[8 * v + 1]) * inv);
+            u.y = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv,
+                                   __uint_as_float(o[8 * v + 3]) * inv);
+            u.z = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv,
+                                   __uint_as_float(o[8 * v + 5]) * inv);
+            u.w = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv,
+                                   __uint_as_float(o[8 * v + 7]) * inv);
+            st_v4(dst + j * 4 + v, u);
+          }
+        }
+      }
+      if (valid && p.lse != nullptr)
+        p.lse[(static_cast<size_t>(b) * p.H + h) * p.L + q_row] =
+            (m + __log2f(lsum)) * 0.69314718055994531f;
+      ptx::tc_fence_before();
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 1) ptx::tmem_dealloc(tmem, T::kTmemCols);
+}
+
+}  // namespace sa

@@ -1,0 +1,625 @@
+// Host side of libsa.so: config validation, the per-tier ring cache manager,
+// the attention plan (attended chunks, slots, relocated temporal bases), RoPE
+// tables, TMA descriptors and kernel launches. See include/sa.h for the
+// contract of each entry point.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "sa_internal.h"
+#include "kernels/attend_simt.cuh"
+#include "kernels/attend_tc.cuh"
+#include "kernels/rope.cuh"
+
+using sa::AttendGroup;
+using sa::AttendParams;
+using sa::AppendParams;
+using sa::RopeTables;
+
+namespace {
+
+thread_local std::string g_error;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Derived {
+  int B, H, D, F, th, tw, S, W, R, L;
+  int dt2, dh2, dw2;
+  float scale, theta;
+  size_t chunk_elems;  // B * H * L * D
+  // byte offsets inside the device buffer
+  size_t off_status, off_rope_t, off_rope_h, off_rope_w, off_tier[2], off_kcur, total;
+};
+
+int validate(const sa_config* c, std::string* why) {
+  auto fail = [&](int code, const char* msg) {
+    if (why) *why = msg;
+    return code;
+  };
+  if (c == nullptr) return fail(SA_ERR_INVALID_ARG, "config is NULL");
+  if (c->batch < 1 || c->heads < 1) return fail(SA_ERR_INVALID_ARG, "batch and heads must be >= 1");
+  if (c->head_dim != 64 && c->head_dim != 128)
+    return fail(SA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (c->frames_per_chunk < 1 || c->tok_h < 1 || c->tok_w < 1)
+    return fail(SA_ERR_INVALID_ARG, "frames_per_chunk, tok_h, tok_w must be >= 1");
+  if (c->sink_chunks < 0 || c->window_chunks < 1)
+    return fail(SA_ERR_INVALID_ARG, "need sink_chunks >= 0 and window_chunks >= 1");
+  if (c->sink_chunks + c->window_chunks > SA_MAX_ATTENDED)
+    return fail(SA_ERR_UNSUPPORTED, "sink_chunks + window_chunks exceeds SA_MAX_ATTENDED");
+  const long long L = 1LL * c->frames_per_chunk * c->tok_h * c->tok_w;
+  if (L > SA_MAX_CHUNK_LEN) return fail(SA_ERR_UNSUPPORTED, "chunk longer than SA_MAX_CHUNK_LEN");
+  if (1LL * c->heads * c->head_dim / 8 > 1024)
+    return fail(SA_ERR_UNSUPPORTED, "heads * head_dim must be <= 8192");
+  if (1LL * c->batch * L > (1LL << 31) - 1) return fail(SA_ERR_UNSUPPORTED, "batch * chunk too big");
+  const long long planes = 2LL * (c->sink_chunks + c->window_chunks) * c->batch * c->heads;
+  if (planes > (1LL << 31) - 1) return fail(SA_ERR_UNSUPPORTED, "too many cache planes");
+  if (!std::isfinite(c->softmax_scale) || !std::isfinite(c->rope_theta))
+    return fail(SA_ERR_INVALID_ARG, "softmax_scale and rope_theta must be finite");
+  return SA_OK;
+}
+
+Derived derive(const sa_config& c) {
+  Derived d{};
+  d.B = c.batch;
+  d.H = c.heads;
+  d.D = c.head_dim;
+  d.F = c.frames_per_chunk;
+  d.th = c.tok_h;
+  d.tw = c.tok_w;
+  d.S = c.sink_chunks;
+  d.W = c.window_chunks;
+  d.R = d.W - 1;
+  d.L = d.F * d.th * d.tw;
+  const int d_sp = 2 * (d.D / 6);
+  d.dt2 = (d.D - 2 * d_sp) / 2;
+  d.dh2 = d_sp / 2;
+  d.dw2 = d_sp / 2;
+  d.scale = c.softmax_scale > 0.f ? c.softmax_scale : 1.f / std::sqrt(static_cast<float>(d.D));
+  d.theta = c.rope_theta > 0.f ? c.rope_theta : 10000.f;
+  d.chunk_elems = static_cast<size_t>(d.B) * d.H * d.L * d.D;
+  const size_t slot_bytes = 2 * d.chunk_elems * sizeof(__nv_bfloat16);
+  size_t off = 0;
+  d.off_status = off;
+  off += 1024;
+  d.off_rope_t = off;
+  off += align_up(static_cast<size_t>(d.S + d.W) * d.F * d.dt2 * sizeof(float2), 1024);
+  d.off_rope_h = off;
+  off += align_up(static_cast<size_t>(d.th) * d.dh2 * sizeof(float2), 1024);
+  d.off_rope_w = off;
+  off += align_up(static_cast<size_t>(d.tw) * d.dw2 * sizeof(float2), 1024);
+  for (int t = 0; t < 2; ++t) {
+    d.off_tier[t] = off;
+    off += align_up(static_cast<size_t>(d.S + d.R) * slot_bytes, 1024);
+  }
+  d.off_kcur = off;
+  off += align_up(d.chunk_elems * sizeof(__nv_bfloat16), 1024);
+  d.total = off;
+  return d;
+}
+
+// Ring slot of chunk `id`: sinks in slots 0..S-1, later chunks in S + (id-S) mod R.
+int slot_of(const Derived& d, int id) {
+  if (id < 0) return -1;
+  if (id < d.S) return id;
+  if (d.R == 0) return -1;
+  return d.S + (id - d.S) % d.R;
+}
+
+// Attended chunks of chunk c, ascending: sinks, the window's cached chunks, c.
+int plan_ids(const Derived& d, int c, int* ids) {
+  int n = 0;
+  for (int j = 0; j < c && j < d.S; ++j) ids[n++] = j;
+  const int lo = c - d.R > d.S ? c - d.R : d.S;
+  for (int j = lo; j < c; ++j) ids[n++] = j;
+  ids[n++] = c;
+  return n;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor whose rows of D elements are tiled by 64-column x `rows` boxes
+// with 128-byte swizzle. dims[0] = D (contiguous); strides in bytes.
+bool encode_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+                const cuuint64_t* strides, const cuuint32_t* box) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
+                  strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// [planes][L][D] with planes contiguous L x D matrices.
+bool encode_planes(CUtensorMap* map, const void* base, const Derived& d, long long planes) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d.D), static_cast<cuuint64_t>(d.L),
+                        static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d.D) * 2,
+                           static_cast<cuuint64_t>(d.L) * d.D * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  return encode_map(map, base, 3, dims, strides, box);
+}
+
+// The caller's [B, L, H, D] tensor as (D, H, L, B).
+bool encode_blhd(CUtensorMap* map, const void* base, const Derived& d) {
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d.D), static_cast<cuuint64_t>(d.H),
+                        static_cast<cuuint64_t>(d.L), static_cast<cuuint64_t>(d.B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(d.D) * 2,
+                           static_cast<cuuint64_t>(d.H) * d.D * 2,
+                           static_cast<cuuint64_t>(d.L) * d.H * d.D * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  return encode_map(map, base, 4, dims, strides, box);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+struct sa_handle {
+  sa_config cfg;
+  Derived d;
+  int device;
+  int sm_count;
+  uint8_t* buf;
+  int count[2];
+  int staged_chunk;  // chunk whose keys sit in the scratch (-1: none)
+  bool has_cache;
+  CUtensorMap tm_tier[2];
+  CUtensorMap tm_kcur;
+  std::string err;
+
+  int fail(int code, const std::string& msg) {
+    err = msg;
+    return code;
+  }
+  unsigned* status() { return reinterpret_cast<unsigned*>(buf + d.off_status); }
+  __nv_bfloat16* tier_base(int t) { return reinterpret_cast<__nv_bfloat16*>(buf + d.off_tier[t]); }
+  __nv_bfloat16* kcur() { return reinterpret_cast<__nv_bfloat16*>(buf + d.off_kcur); }
+  RopeTables rope() {
+    RopeTables rt;
+    rt.t = reinterpret_cast<const float2*>(buf + d.off_rope_t);
+    rt.h = reinterpret_cast<const float2*>(buf + d.off_rope_h);
+    rt.w = reinterpret_cast<const float2*>(buf + d.off_rope_w);
+    rt.dt2 = d.dt2;
+    rt.dh2 = d.dh2;
+    rt.dw2 = d.dw2;
+    rt.tok_h = d.th;
+    rt.tok_w = d.tw;
+    rt.frame_tokens = d.th * d.tw;
+    return rt;
+  }
+};
+
+namespace {
+
+int check_device(sa_handle* h) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return h->fail(SA_ERR_CUDA, "cudaGetDevice failed");
+  if (dev != h->device)
+    return h->fail(SA_ERR_INVALID_ARG, "current device differs from the handle's device");
+  return SA_OK;
+}
+
+int launch_rope_transpose(sa_handle* h, const void* K, const void* V, __nv_bfloat16* k_out,
+                          __nv_bfloat16* v_out, cudaStream_t s) {
+  const Derived& d = h->d;
+  AppendParams ap;
+  ap.k_in = static_cast<const __nv_bfloat16*>(K);
+  ap.v_in = static_cast<const __nv_bfloat16*>(V);
+  ap.k_out = k_out;
+  ap.v_out = v_out;
+  ap.B = d.B;
+  ap.L = d.L;
+  ap.H = d.H;
+  ap.D = d.D;
+  ap.rope = h->rope();
+  const int threads = static_cast<int>(align_up(static_cast<size_t>(d.H) * d.D / 8, 32));
+  dim3 grid(static_cast<unsigned>(d.B) * d.L, V != nullptr ? 2 : 1);
+  sa::rope_transpose_kernel<<<grid, threads, 0, s>>>(ap);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return h->fail(SA_ERR_CUDA, std::string("append launch: ") + cudaGetErrorString(e));
+  return SA_OK;
+}
+
+int check_handle(sa_handle* h) {
+  if (h == nullptr) {
+    g_error = "handle is NULL";
+    return SA_ERR_INVALID_ARG;
+  }
+  return SA_OK;
+}
+
+int stage_keys(sa_handle* h, const void* Kc, sa_stream stream) {
+  int rc = check_handle(h);
+  if (rc != SA_OK) return rc;
+  if (Kc == nullptr || !aligned16(Kc))
+    return h->fail(SA_ERR_INVALID_ARG, "Kc must be a non-NULL 16-byte aligned pointer");
+  if (h->count[0] != h->count[1])
+    return h->fail(SA_ERR_STATE, "both tiers must hold the same chunks before attending");
+  rc = check_device(h);
+  if (rc != SA_OK) return rc;
+  rc = launch_rope_transpose(h, Kc, nullptr, h->kcur(), nullptr,
+                             reinterpret_cast<cudaStream_t>(stream));
+  if (rc != SA_OK) return rc;
+  h->staged_chunk = h->count[0];
+  return SA_OK;
+}
+
+int attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final, void* O,
+                  float* lse, sa_stream stream, bool simt) {
+  int rc = check_handle(h);
+  if (rc != SA_OK) return rc;
+  if (Q == nullptr || Vc == nullptr || O == nullptr)
+    return h->fail(SA_ERR_INVALID_ARG, "Q, Vc and O must be non-NULL");
+  if (!aligned16(Q) || !aligned16(Vc) || !aligned16(O))
+    return h->fail(SA_ERR_INVALID_ARG, "Q, Vc and O must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+    return h->fail(SA_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+  if (O == Q || O == Vc) return h->fail(SA_ERR_INVALID_ARG, "O must not alias an input");
+  if (h->count[0] != h->count[1])
+    return h->fail(SA_ERR_STATE, "both tiers must hold the same chunks before attending");
+  if (h->staged_chunk != h->count[0])
+    return h->fail(SA_ERR_STATE, "no keys staged for the current chunk (call sa_stage_keys)");
+  rc = check_device(h);
+  if (rc != SA_OK) return rc;
+  const Derived& d = h->d;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int tier = step_is_final ? SA_TIER_CLEAN : SA_TIER_NOISY;
+  const int c = h->count[0];
+
+  AttendParams ap;
+  std::memset(&ap, 0, sizeof(ap));
+  ap.q = static_cast<const __nv_bfloat16*>(Q);
+  ap.o = static_cast<__nv_bfloat16*>(O);
+  ap.lse = lse;
+  ap.cache = h->tier_base(tier);
+  ap.k_cur = h->kcur();
+  ap.v_cur = static_cast<const __nv_bfloat16*>(Vc);
+  ap.B = d.B;
+  ap.L = d.L;
+  ap.H = d.H;
+  ap.D = d.D;
+  int ids[SA_MAX_ATTENDED];
+  const int n = plan_ids(d, c, ids);
+  ap.n_groups = n;
+  for (int g = 0; g < n; ++g) {
+    AttendGroup& grp = ap.groups[g];
+    grp.src = ids[g] == c ? 1 : 0;
+    grp.slot = ids[g] == c ? 0 : slot_of(d, ids[g]);
+    grp.t_delta = (n - 1 - g) * d.F;
+    grp.len = d.L;
+  }
+  ap.scale_log2 = d.scale * 1.4426950408889634f;
+  ap.rope = h->rope();
+  ap.status = h->status();
+
+  if (simt) {
+    const long long rows = 1LL * d.B * d.H * d.L;
+    const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
+    if (d.D == 128)
+      sa::attend_simt_kernel<128><<<grid, 256, 0, s>>>(ap);
+    else
+      sa::attend_simt_kernel<64><<<grid, 256, 0, s>>>(ap);
+  } else {
+    CUtensorMap tm_v;
+    if (!encode_blhd(&tm_v, Vc, d)) return h->fail(SA_ERR_CUDA, "TMA descriptor for Vc failed");
+    const CUtensorMap& tm_cache = h->has_cache ? h->tm_tier[tier] : h->tm_kcur;
+    const int n_qt = (d.L + 127) / 128;
+    const long long n_work = 1LL * d.B * d.H * ((n_qt + 1) / 2);
+    const unsigned grid = static_cast<unsigned>(n_work < h->sm_count ? n_work : h->sm_count);
+    if (d.D == 128)
+      sa::attend_tc_kernel<128><<<grid, sa::TcShape<128>::kThreads, sa::TcShape<128>::kSmemBytes,
+                                  s>>>(tm_cache, h->tm_kcur, tm_v, ap);
+    else
+      sa::attend_tc_kernel<64><<<grid, sa::TcShape<64>::kThreads, sa::TcShape<64>::kSmemBytes,
+                                 s>>>(tm_cache, h->tm_kcur, tm_v, ap);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return h->fail(SA_ERR_CUDA, std::string("attend launch: ") + cudaGetErrorString(e));
+  return SA_OK;
+}
+
+int attend_common(sa_handle* h, const void* Q, const void* Kc, const void* Vc, int step_is_final,
+                  void* O, float* lse, sa_stream stream, bool simt) {
+  int rc = check_handle(h);
+  if (rc != SA_OK) return rc;
+  if (Q == nullptr || Kc == nullptr || Vc == nullptr || O == nullptr)
+    return h->fail(SA_ERR_INVALID_ARG, "Q, Kc, Vc and O must be non-NULL");
+  if (O == Kc) return h->fail(SA_ERR_INVALID_ARG, "O must not alias an input");
+  // Validate the attention half before launching the staging half.
+  if (!aligned16(Q) || !aligned16(Vc) || !aligned16(O) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 || O == Q || O == Vc)
+    return h->fail(SA_ERR_INVALID_ARG, "Q, Vc, O must be 16-byte aligned, lse 4-byte aligned, "
+                                       "O must not alias an input");
+  rc = stage_keys(h, Kc, stream);
+  if (rc != SA_OK) return rc;
+  return attend_staged(h, Q, Vc, step_is_final, O, lse, stream, simt);
+}
+
+}  // namespace
+
+extern "C" {
+
+SA_API int sa_validate_config(const sa_config* cfg) {
+  std::string why;
+  int rc = validate(cfg, &why);
+  if (rc != SA_OK) g_error = why;
+  return rc;
+}
+
+SA_API size_t sa_required_bytes(const sa_config* cfg) {
+  if (sa_validate_config(cfg) != SA_OK) return 0;
+  return derive(*cfg).total;
+}
+
+SA_API int sa_create(const sa_config* cfg, void* dev_buf, size_t bytes, sa_handle** out) {
+  if (out == nullptr) {
+    g_error = "out is NULL";
+    return SA_ERR_INVALID_ARG;
+  }
+  *out = nullptr;
+  std::string why;
+  int rc = validate(cfg, &why);
+  if (rc != SA_OK) {
+    g_error = why;
+    return rc;
+  }
+  const Derived d = derive(*cfg);
+  if (dev_buf == nullptr || (reinterpret_cast<uintptr_t>(dev_buf) & 255u) != 0) {
+    g_error = "dev_buf must be a non-NULL, 256-byte aligned device pointer";
+    return SA_ERR_INVALID_ARG;
+  }
+  if (bytes < d.total) {
+    g_error = "dev_buf smaller than sa_required_bytes(cfg)";
+    return SA_ERR_INVALID_ARG;
+  }
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, dev_buf) != cudaSuccess || attr.type != cudaMemoryTypeDevice) {
+    cudaGetLastError();
+    g_error = "dev_buf is not device memory";
+    return SA_ERR_INVALID_ARG;
+  }
+  int dev = -1, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || attr.device != dev) {
+    g_error = "dev_buf is not on the current device";
+    return SA_ERR_INVALID_ARG;
+  }
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (major != 10 || minor != 0) {
+    g_error = "this library is built for sm_100a (B200) only";
+    return SA_ERR_UNSUPPORTED;
+  }
+
+  sa_handle* h = new sa_handle();
+  h->cfg = *cfg;
+  h->d = d;
+  h->device = dev;
+  h->sm_count = sms;
+  h->buf = static_cast<uint8_t*>(dev_buf);
+  h->count[0] = h->count[1] = 0;
+  h->staged_chunk = -1;
+
+  // RoPE tables: angle pos * theta^(-2i/d) in double, cos/sin cast to float.
+  std::vector<float2> t(static_cast<size_t>(d.S + d.W) * d.F * d.dt2);
+  std::vector<float2> th(static_cast<size_t>(d.th) * d.dh2), tw(static_cast<size_t>(d.tw) * d.dw2);
+  auto fill = [&](std::vector<float2>& tab, int npos, int npair) {
+    const double band = 2.0 * npair;
+    for (int pos = 0; pos < npos; ++pos)
+      for (int i = 0; i < npair; ++i) {
+        const double a = pos * std::pow(static_cast<double>(d.theta), -2.0 * i / band);
+        tab[static_cast<size_t>(pos) * npair + i] =
+            make_float2(static_cast<float>(std::cos(a)), static_cast<float>(std::sin(a)));
+      }
+  };
+  fill(t, (d.S + d.W) * d.F, d.dt2);
+  fill(th, d.th, d.dh2);
+  fill(tw, d.tw, d.dw2);
+  bool ok = cudaMemset(h->buf + d.off_status, 0, 1024) == cudaSuccess;
+  ok = ok && cudaMemcpy(h->buf + d.off_rope_t, t.data(), t.size() * sizeof(float2),
+                        cudaMemcpyHostToDevice) == cudaSuccess;
+  ok = ok && cudaMemcpy(h->buf + d.off_rope_h, th.data(), th.size() * sizeof(float2),
+                        cudaMemcpyHostToDevice) == cudaSuccess;
+  ok = ok && cudaMemcpy(h->buf + d.off_rope_w, tw.data(), tw.size() * sizeof(float2),
+                        cudaMemcpyHostToDevice) == cudaSuccess;
+  if (!ok) {
+    g_error = std::string("uploading RoPE tables failed: ") + cudaGetErrorString(cudaGetLastError());
+    delete h;
+    return SA_ERR_CUDA;
+  }
+  h->has_cache = d.S + d.R > 0;
+  if (h->has_cache) {
+    for (int tier = 0; tier < 2; ++tier)
+      if (!encode_planes(&h->tm_tier[tier], h->tier_base(tier), d, 2LL * (d.S + d.R) * d.B * d.H)) {
+        g_error = "TMA descriptor for the cache failed";
+        delete h;
+        return SA_ERR_CUDA;
+      }
+  }
+  if (!encode_planes(&h->tm_kcur, h->kcur(), d, 1LL * d.B * d.H)) {
+    g_error = "TMA descriptor for the key scratch failed";
+    delete h;
+    return SA_ERR_CUDA;
+  }
+  cudaError_t e = cudaFuncSetAttribute(sa::attend_tc_kernel<128>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       sa::TcShape<128>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(sa::attend_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sa::TcShape<64>::kSmemBytes);
+  if (e != cudaSuccess) {
+    g_error = std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e);
+    delete h;
+    return SA_ERR_CUDA;
+  }
+  *out = h;
+  return SA_OK;
+}
+
+SA_API int sa_destroy(sa_handle* h) {
+  delete h;
+  return SA_OK;
+}
+
+SA_API int sa_reset(sa_handle* h) {
+  if (h == nullptr) {
+    g_error = "handle is NULL";
+    return SA_ERR_INVALID_ARG;
+  }
+  int rc = check_device(h);
+  if (rc != SA_OK) return rc;
+  h->count[0] = h->count[1] = 0;
+  h->staged_chunk = -1;
+  if (cudaMemset(h->buf + h->d.off_status, 0, 1024) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess)
+    return h->fail(SA_ERR_CUDA, "clearing the status word failed");
+  return SA_OK;
+}
+
+SA_API int sa_append_chunk(sa_handle* h, int tier, const void* K, const void* V,
+                           sa_stream stream) {
+  if (h == nullptr) {
+    g_error = "handle is NULL";
+    return SA_ERR_INVALID_ARG;
+  }
+  if (tier != SA_TIER_NOISY && tier != SA_TIER_CLEAN)
+    return h->fail(SA_ERR_INVALID_ARG, "tier must be SA_TIER_NOISY or SA_TIER_CLEAN");
+  if (K == nullptr || V == nullptr) return h->fail(SA_ERR_INVALID_ARG, "K and V must be non-NULL");
+  if (!aligned16(K) || !aligned16(V))
+    return h->fail(SA_ERR_INVALID_ARG, "K and V must be 16-byte aligned");
+  if (h->count[tier] > h->count[1 - tier])
+    return h->fail(SA_ERR_STATE, "this tier is already one chunk ahead of the other");
+  int rc = check_device(h);
+  if (rc != SA_OK) return rc;
+  const int id = h->count[tier];
+  const int slot = slot_of(h->d, id);
+  if (slot >= 0) {
+    __nv_bfloat16* base = h->tier_base(tier) + static_cast<size_t>(slot) * 2 * h->d.chunk_elems;
+    rc = launch_rope_transpose(h, K, V, base, base + h->d.chunk_elems,
+                               reinterpret_cast<cudaStream_t>(stream));
+    if (rc != SA_OK) return rc;
+  }
+  h->count[tier] = id + 1;
+  return SA_OK;
+}
+
+SA_API int sa_attend(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
+                     int step_is_final, void* O, float* lse, sa_stream stream) {
+  return attend_common(h, Q, Kc, Vc, step_is_final, O, lse, stream, false);
+}
+
+SA_API int sa_stage_keys(sa_handle* h, const void* Kc, sa_stream stream) {
+  return stage_keys(h, Kc, stream);
+}
+
+SA_API int sa_attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final,
+                            void* O, float* lse, sa_stream stream) {
+  return attend_staged(h, Q, Vc, step_is_final, O, lse, stream, false);
+}
+
+SA_API int sa_debug_attend_simt(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
+                                int step_is_final, void* O, float* lse, sa_stream stream) {
+  return attend_common(h, Q, Kc, Vc, step_is_final, O, lse, stream, true);
+}
+
+SA_API int sa_chunk_count(const sa_handle* h, int tier) {
+  if (h == nullptr || (tier != SA_TIER_NOISY && tier != SA_TIER_CLEAN)) return -SA_ERR_INVALID_ARG;
+  return h->count[tier];
+}
+
+SA_API int sa_debug_layout(const sa_handle* h, int tier, int32_t* slot_chunk_ids, int n) {
+  if (h == nullptr || slot_chunk_ids == nullptr || (tier != SA_TIER_NOISY && tier != SA_TIER_CLEAN))
+    return -SA_ERR_INVALID_ARG;
+  const Derived& d = h->d;
+  const int slots = d.S + d.R;
+  const int m = n < slots ? n : slots;
+  for (int s = 0; s < m; ++s) slot_chunk_ids[s] = -1;
+  const int cnt = h->count[tier];
+  for (int j = 0; j < cnt; ++j) {  // the latest chunk written to a slot holds it
+    const int s = slot_of(d, j);
+    if (s >= 0 && s < m) slot_chunk_ids[s] = j;
+  }
+  return m;
+}
+
+SA_API int sa_plan(const sa_config* cfg, int32_t chunk, int32_t* ids, int32_t* slots,
+                   int32_t* t_base, int cap) {
+  std::string why;
+  if (validate(cfg, &why) != SA_OK || chunk < 0) {
+    g_error = chunk < 0 ? "chunk must be >= 0" : why;
+    return -SA_ERR_INVALID_ARG;
+  }
+  const Derived d = derive(*cfg);
+  int tmp[SA_MAX_ATTENDED];
+  const int n = plan_ids(d, chunk, tmp);
+  if (cap < n) {
+    g_error = "cap too small";
+    return -SA_ERR_INVALID_ARG;
+  }
+  for (int g = 0; g < n; ++g) {
+    if (ids) ids[g] = tmp[g];
+    if (slots) slots[g] = tmp[g] == chunk ? -1 : slot_of(d, tmp[g]);
+    if (t_base) t_base[g] = g * d.F;
+  }
+  return n;
+}
+
+SA_API int sa_slot_of(const sa_config* cfg, int32_t chunk) {
+  if (validate(cfg, nullptr) != SA_OK) return -1;
+  return slot_of(derive(*cfg), chunk);
+}
+
+SA_API int sa_get_status(sa_handle* h, sa_stream stream) {
+  if (h == nullptr) {
+    g_error = "handle is NULL";
+    return SA_ERR_INVALID_ARG;
+  }
+  unsigned word = 0;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess ||
+      cudaMemcpy(&word, h->status(), sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return h->fail(SA_ERR_CUDA, std::string("reading the status word: ") +
+                                    cudaGetErrorString(cudaGetLastError()));
+  if (word & sa::kDevErrTimeout) return h->fail(SA_ERR_TIMEOUT, "a kernel gave up a bounded wait");
+  return SA_OK;
+}
+
+SA_API const char* sa_last_error(const sa_handle* h) {
+  return h != nullptr ? h->err.c_str() : g_error.c_str();
+}
+
+SA_API const char* sa_status_string(int status) {
+  switch (status) {
+    case SA_OK: return "SA_OK";
+    case SA_ERR_INVALID_ARG: return "SA_ERR_INVALID_ARG";
+    case SA_ERR_STATE: return "SA_ERR_STATE";
+    case SA_ERR_UNSUPPORTED: return "SA_ERR_UNSUPPORTED";
+    case SA_ERR_CUDA: return "SA_ERR_CUDA";
+    case SA_ERR_TIMEOUT: return "SA_ERR_TIMEOUT";
+    default: return "SA_ERR_UNKNOWN";
+  }
+}
+
+}  // extern "C"

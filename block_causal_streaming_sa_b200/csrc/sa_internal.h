@@ -1,0 +1,63 @@
+// Internal types shared by the host side (sa_api.cu) and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "../../include/sa.h"
+
+namespace sa {
+
+constexpr int kMaxGroups = SA_MAX_ATTENDED;
+
+// Device status word bits (written with atomicOr, read by sa_get_status).
+constexpr unsigned kDevErrTimeout = 1u;
+
+// fp32 (cos, sin) tables of the three RoPE bands (reading: bands [t | h | w] of
+// D - 4*(D/6), 2*(D/6), 2*(D/6) dims, pair i of a band of size d turned by
+// pos * theta^(-2i/d)). Row = position, column = pair index in the band.
+struct RopeTables {
+  const float2* t;  // [(S + W) * F][dt2]
+  const float2* h;  // [tok_h][dh2]
+  const float2* w;  // [tok_w][dw2]
+  int dt2, dh2, dw2;
+  int tok_h, tok_w, frame_tokens;  // frame_tokens = tok_h * tok_w
+};
+
+// Rotate-and-transpose of one chunk: in [B, L, H, D] -> out [B, H, L, D].
+// K rows are turned by their in-chunk (frame, row, column) position; V rows
+// (blockIdx.y == 1) are copied.
+struct AppendParams {
+  const __nv_bfloat16* k_in;
+  const __nv_bfloat16* v_in;  // may be null (K only)
+  __nv_bfloat16* k_out;
+  __nv_bfloat16* v_out;
+  int B, L, H, D;
+  RopeTables rope;
+};
+
+// One attended chunk, in ascending chunk-id order.
+struct AttendGroup {
+  int src;      // 0: cache slot of the selected tier, 1: the chunk being generated
+  int slot;     // cache slot (src == 0)
+  int t_delta;  // (rank(current) - rank(this chunk)) * F, >= 0
+  int len;      // number of keys
+};
+
+struct AttendParams {
+  const __nv_bfloat16* q;        // [B, L, H, D] unrotated
+  __nv_bfloat16* o;              // [B, L, H, D]
+  float* lse;                    // [B, H, L] or null
+  const __nv_bfloat16* cache;    // selected tier: [slot][K|V][B][H][L][D], K rotated in-chunk
+  const __nv_bfloat16* k_cur;    // current chunk K, rotated in-chunk: [B][H][L][D]
+  const __nv_bfloat16* v_cur;    // current chunk V as passed: [B][L][H][D]
+  int B, L, H, D;
+  int n_groups;
+  AttendGroup groups[kMaxGroups];
+  float scale_log2;  // softmax scale * log2(e)
+  RopeTables rope;
+  unsigned* status;
+};
+
+}  // namespace sa

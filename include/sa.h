@@ -1,0 +1,186 @@
+/*
+ * sa.h - C ABI of the block-causal streaming attention library (libsa.so).
+ *
+ * One chunk's attention over a bounded two-tier KV cache of sink chunks plus a
+ * rolling window of recent chunks, with relocated temporal RoPE, on NVIDIA B200
+ * (sm_100a).
+ *
+ * Where the operation is defined (web pages, cited by title and section):
+ *  - "Vidu S2 vs PixVerse R2：实时视频的两条技术路线" (orkas.ai blog):
+ *      section 「实时」改变了什么 - video is generated chunk by chunk in order; a
+ *      chunk sees what came before it, never what comes after (block causal).
+ *      section 选择三：有上限的记忆 - the first chunks are kept for good as anchors
+ *      (sink), a sliding window of the most recent chunks is kept and older ones
+ *      are dropped; temporal positions are relocated into the trained range
+ *      ("RoPE relocation"); TwinCache caches every history chunk twice, noisy and
+ *      clean: intermediate denoising steps read the noisy copy, the final step
+ *      reads the clean copy.
+ *  - "Vidu S2：实时可交互、可编辑、可立体的视频生成" (paper read of Vidu S2):
+ *      abbreviation table - the KV cache stores history keys and values so they
+ *      are not recomputed; RoPE encodes each token's position in space and time.
+ *      section 2.2 - block-wise causal mask, anchor chunks, sliding-window
+ *      context, noisy KV cache.
+ *
+ * Conventions shared by every call
+ *  - Tensors are bfloat16, row-major [B, L, H, D] (batch, token of the chunk,
+ *    head, head dim), contiguous, 16-byte aligned, in device memory of the
+ *    device the handle was created on. Token l of a chunk is frame
+ *    l / (tok_h * tok_w), row (l / tok_w) % tok_h, column l % tok_w.
+ *  - K and V passed in are UNROTATED; the library applies the 3D RoPE.
+ *  - All device work is asynchronous on the caller's stream (a cudaStream_t
+ *    passed as sa_stream; NULL is the legacy default stream). After sa_create,
+ *    sa_append_chunk / sa_stage_keys / sa_attend_staged / sa_attend allocate no
+ *    memory and never synchronise the host.
+ *  - Every call returns an sa_status. On error nothing is launched and the
+ *    handle's counters are unchanged; sa_last_error() explains the failure.
+ *  - A handle is not thread-safe: one host thread drives one handle.
+ */
+#ifndef BLOCK_CAUSAL_STREAMING_SA_H
+#define BLOCK_CAUSAL_STREAMING_SA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SA_API __attribute__((visibility("default")))
+
+typedef struct sa_handle sa_handle;
+typedef void* sa_stream; /* a cudaStream_t */
+
+typedef enum {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or config field */
+  SA_ERR_STATE = 2,        /* call not allowed in the handle's current state */
+  SA_ERR_UNSUPPORTED = 3,  /* valid request this build cannot serve (e.g. D) */
+  SA_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed */
+  SA_ERR_TIMEOUT = 5       /* a kernel gave up a bounded wait (device status) */
+} sa_status;
+
+typedef enum { SA_TIER_NOISY = 0, SA_TIER_CLEAN = 1 } sa_tier;
+
+/* Shape of one attention layer's stream. */
+typedef struct {
+  int32_t batch;            /* B >= 1 */
+  int32_t heads;            /* H >= 1 */
+  int32_t head_dim;         /* D: 64 or 128 */
+  int32_t frames_per_chunk; /* F >= 1 latent frames per chunk */
+  int32_t tok_h, tok_w;     /* tokens per frame: rows x columns */
+  int32_t sink_chunks;      /* S >= 0 chunks kept for good */
+  int32_t window_chunks;    /* W >= 1 most recent chunks attended, counting the
+                               chunk being generated; W - 1 are cached */
+  float softmax_scale;      /* <= 0 selects 1/sqrt(D) */
+  float rope_theta;         /* <= 0 selects 10000 */
+} sa_config;
+
+/* Upper bounds of this build (checked by sa_validate_config). */
+#define SA_MAX_ATTENDED 16 /* S + W */
+#define SA_MAX_CHUNK_LEN (1 << 22)
+
+/* Validate a config; SA_OK or SA_ERR_INVALID_ARG / SA_ERR_UNSUPPORTED. Host only. */
+SA_API int sa_validate_config(const sa_config* cfg);
+
+/* Bytes of device memory sa_create needs for cfg (0 if cfg is invalid):
+ * a status word, fp32 RoPE tables, both cache tiers ((S + W - 1) slots of K and
+ * V each, layout [slot][K|V][B][H][L][D]) and one rotated-key chunk of scratch
+ * for the chunk being generated. Host only. */
+SA_API size_t sa_required_bytes(const sa_config* cfg);
+
+/* Create a handle over a caller-owned device buffer of at least
+ * sa_required_bytes(cfg) bytes, 256-byte aligned, on the current device.
+ * Writes the RoPE tables into it (synchronously) and encodes the TMA
+ * descriptors of the cache. The buffer stays owned by the caller and must
+ * outlive the handle. Returns SA_OK and *out, or an error and *out = NULL. */
+SA_API int sa_create(const sa_config* cfg, void* dev_buf, size_t bytes, sa_handle** out);
+
+/* Release the handle (host memory only; the caller frees dev_buf). NULL is OK. */
+SA_API int sa_destroy(sa_handle* h);
+
+/* Forget every cached chunk and clear the device status word (start a new
+ * stream). Enqueues one small memset on the default stream of the device and
+ * waits for it; not for use inside graph capture. */
+SA_API int sa_reset(sa_handle* h);
+
+/* Append the next chunk's K/V ([B, L, H, D], unrotated) to one tier.
+ * Chunk ids count from 0 per tier. Chunk id n goes to slot n if n < S, else to
+ * window slot S + (n - S) mod (W - 1), overwriting (evicting) the oldest
+ * non-sink chunk once the window is full; with W == 1 a non-sink chunk is not
+ * stored. K is rotated by its in-chunk (frame, row, column) position on the way
+ * in; the relocated temporal offset is applied at attend time.
+ * A tier may run at most one chunk ahead of the other: appending to the tier
+ * that is already ahead is SA_ERR_STATE. K and V may be freed once the launch
+ * on `stream` has run. */
+SA_API int sa_append_chunk(sa_handle* h, int tier, const void* K, const void* V,
+                           sa_stream stream);
+
+/* Attention of the chunk being generated (chunk id c = number of chunks in
+ * both tiers) at one denoising step:
+ *   O = softmax(rope(Q) rope(K)^T * scale) V
+ * over the keys of every cached sink and window chunk of the selected tier
+ * (clean if step_is_final != 0, else noisy) followed by the chunk's own Kc/Vc,
+ * all bidirectional inside the chunk. Chunk j sits at temporal position
+ * rank(j) * F + frame, rank = index of j among the attended chunks in
+ * ascending id order, so positions stay below (S + W) * F.
+ * Q, Kc, Vc: [B, L, H, D] bf16 (unrotated), read only.
+ * O: [B, L, H, D] bf16, fully overwritten (must not alias the inputs).
+ * lse: optional [B, H, L] fp32 natural-log sum of exp of the scaled scores
+ *      (NULL to skip), for merging partial attentions.
+ * Requires both tiers to hold the same number of chunks (else SA_ERR_STATE).
+ * Uses the handle's rotated-key scratch: calls on one handle must be ordered
+ * on the GPU (same stream, or events). */
+SA_API int sa_attend(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
+                     int step_is_final, void* O, float* lse, sa_stream stream);
+
+/* The two halves of sa_attend, for callers that time or schedule them apart.
+ * sa_stage_keys rotates the generating chunk's Kc ([B, L, H, D] bf16) by its
+ * in-chunk positions into the handle's key scratch (one HBM-bound kernel).
+ * sa_attend_staged then runs the attention kernel over the cache and the staged
+ * keys, with Vc read in place. sa_attend_staged requires a preceding
+ * sa_stage_keys for the same chunk (else SA_ERR_STATE); the staged keys stay
+ * valid until the next sa_stage_keys / sa_attend on this handle. */
+SA_API int sa_stage_keys(sa_handle* h, const void* Kc, sa_stream stream);
+SA_API int sa_attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final,
+                            void* O, float* lse, sa_stream stream);
+
+/* Same contract as sa_attend, computed by a plain fp32 SIMT kernel (one warp
+ * per query row, no tensor cores). A debugging cross-check of the tensor-core
+ * kernel, an order of magnitude slower; not used by sa_attend. */
+SA_API int sa_debug_attend_simt(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
+                                int step_is_final, void* O, float* lse, sa_stream stream);
+
+/* Chunks appended so far to `tier`, or a negative sa_status. */
+SA_API int sa_chunk_count(const sa_handle* h, int tier);
+
+/* Chunk id held by each slot of `tier` (-1 = empty), for the first
+ * min(n, S + W - 1) slots; returns the number of slots written. Host only. */
+SA_API int sa_debug_layout(const sa_handle* h, int tier, int32_t* slot_chunk_ids, int n);
+
+/* The attention plan of chunk `chunk` of a stream with config cfg, computed on
+ * the host with no handle and no device: writes, for each attended chunk in
+ * ascending id order, its id, its cache slot (-1 for the chunk itself) and its
+ * relocated temporal base rank * F. Returns the count (<= S + W) or a negative
+ * sa_status if cap is too small. */
+SA_API int sa_plan(const sa_config* cfg, int32_t chunk, int32_t* ids, int32_t* slots,
+                   int32_t* t_base, int cap);
+
+/* Slot of chunk id `chunk` in a tier (-1 if it is never stored). Host only. */
+SA_API int sa_slot_of(const sa_config* cfg, int32_t chunk);
+
+/* Wait for `stream`, then read and return the device status word: SA_OK, or
+ * SA_ERR_TIMEOUT if a kernel gave up a bounded wait since the last reset. */
+SA_API int sa_get_status(sa_handle* h, sa_stream stream);
+
+/* Text of the handle's last error (never NULL); with h == NULL, of the last
+ * error of a call that had no handle yet (sa_create). */
+SA_API const char* sa_last_error(const sa_handle* h);
+
+/* Name of an sa_status value. */
+SA_API const char* sa_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BLOCK_CAUSAL_STREAMING_SA_H */

@@ -14,6 +14,8 @@ function of (seed, shape) and can be re-drawn anywhere.
 """
 
 import hashlib
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -41,13 +43,35 @@ def uniforms(seed, start, count):
     return (z >> np.uint64(11)).astype(np.float64) * (1.0 / (1 << 53))
 
 
+_POOL = None
+
+
+def _pool():
+    global _POOL
+    if _POOL is None:
+        _POOL = ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1))
+    return _POOL
+
+
+def _blocks(count, fn):
+    """Run fn(start, n) over blocks of the index range (threads; numpy drops the GIL)."""
+    starts = range(0, count, _BLOCK)
+    if count <= _BLOCK:
+        for s in starts:
+            fn(s, min(_BLOCK, count - s))
+        return
+    list(_pool().map(lambda s: fn(s, min(_BLOCK, count - s)), starts))
+
+
 def normals(seed, count):
     """``count`` standard normal float64 values of stream ``seed``."""
     out = np.empty(count, dtype=np.float64)
-    for s in range(0, count, _BLOCK):
-        n = min(_BLOCK, count - s)
+
+    def fill(s, n):
         u = uniforms(seed, 2 * s, 2 * n)
         out[s:s + n] = np.sqrt(-2.0 * np.log1p(-u[0::2])) * np.cos(2.0 * np.pi * u[1::2])
+
+    _blocks(count, fill)
     return out
 
 
@@ -61,13 +85,20 @@ def normal_bf16(seed, shape, scale=1.0, outlier_frac=0.0, outlier_mag=8.0):
     """bf16 CPU tensor of N(0, scale^2) values; optionally a Bernoulli
     ``outlier_frac`` share of elements replaced by +-``outlier_mag``."""
     count = int(np.prod(shape))
-    vals = normals(seed, count) * scale
-    if outlier_frac > 0.0:
-        pick = uniforms(seed_of(seed, "outlier"), 0, count) < outlier_frac
-        sign = np.where(uniforms(seed_of(seed, "sign"), 0, count) < 0.5, -1.0, 1.0)
-        vals = np.where(pick, sign * outlier_mag, vals)
-    t = torch.from_numpy(vals.astype(np.float32).reshape(shape))
-    return t.to(torch.bfloat16)
+    vals = normals(seed, count)
+    out = np.empty(count, dtype=np.float32)
+    s_pick, s_sign = seed_of(seed, "outlier"), seed_of(seed, "sign")
+
+    def fill(s, n):
+        v = vals[s:s + n] * scale
+        if outlier_frac > 0.0:
+            pick = uniforms(s_pick, s, n) < outlier_frac
+            sign = np.where(uniforms(s_sign, s, n) < 0.5, -1.0, 1.0)
+            v = np.where(pick, sign * outlier_mag, v)
+        out[s:s + n] = v
+
+    _blocks(count, fill)
+    return torch.from_numpy(out.reshape(shape)).to(torch.bfloat16)
 
 
 @dataclass(frozen=True)

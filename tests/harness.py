@@ -1,0 +1,82 @@
+"""Drives the CUDA library and the oracle with the same seeded inputs.
+
+Test infrastructure: the library is called through its C ABI (ctypes binding),
+the oracle in float64 on the CPU; only the seeded inputs are shared.
+"""
+
+import numpy as np
+import torch
+
+import block_causal_streaming_sa_b200 as sa
+from oracle.stream import CLEAN, NOISY, OracleConfig, StreamOracle
+
+TOL = 1e-2  # max |O_gpu - O_oracle| on bf16 outputs with fp32 accumulation
+
+
+def f64(t):
+    return t.to(torch.float64).numpy()
+
+
+def sample_rows(L, n, seed):
+    """n seeded query rows including the first, the last and tile edges."""
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, L - 1] + [r for r in (127, 128, 255, 256) if r < L]
+    rest = rng.choice(L, size=min(L, n), replace=False)
+    return np.unique(np.concatenate([fixed, rest]))
+
+
+class Pair:
+    """One library handle and one oracle stream fed the same chunks.
+
+    ``batches``/``heads`` restrict what the oracle stores and computes (it works
+    per (b, h), so slicing its inputs is exact); the library always gets the
+    full tensors.
+    """
+
+    def __init__(self, w, batches=None, heads=None, layer=0):
+        self.w = w
+        self.layer = layer
+        self.gpu = sa.StreamingAttention(w.config_dict())
+        self.bsel = list(range(w.batch)) if batches is None else list(batches)
+        self.hsel = list(range(w.heads)) if heads is None else list(heads)
+        self.ocfg = OracleConfig(len(self.bsel), len(self.hsel), w.head_dim, w.frames,
+                                 w.tok_h, w.tok_w, w.sink, w.window)
+        self.oracle = StreamOracle(self.ocfg)
+        self.chunk = 0
+
+    def _slice(self, t):
+        return f64(t)[self.bsel][:, :, self.hsel]
+
+    def tensors(self, names, step=0, chunk=None):
+        c = self.chunk if chunk is None else chunk
+        return [self.w.tensor(n, c, step, self.layer) for n in names]
+
+    def append(self, tensors=None):
+        """Append the current chunk's noisy and clean K/V to both sides."""
+        Kn, Vn, Kcl, Vcl = tensors if tensors is not None else self.tensors(
+            ("Kn", "Vn", "Kcl", "Vcl"))
+        for tier, K, V in ((NOISY, Kn, Vn), (CLEAN, Kcl, Vcl)):
+            self.gpu.append(tier, K.cuda(), V.cuda())
+            self.oracle.append(tier, self._slice(K), self._slice(V))
+        self.chunk += 1
+
+    def attend(self, step, final, rows=None, simt=False, tensors=None):
+        """(O_gpu [B', rows, H', D] float64, O_oracle, lse_gpu, lse_oracle)."""
+        Q, Kc, Vc = tensors if tensors is not None else self.tensors(("Q", "Kc", "Vc"), step)
+        b, l, h, _ = Q.shape
+        lse = torch.empty((b, h, l), dtype=torch.float32, device="cuda")
+        out = self.gpu.attend(Q.cuda(), Kc.cuda(), Vc.cuda(), final, lse=lse, simt=simt)
+        torch.cuda.synchronize()
+        rows_idx = np.arange(l) if rows is None else np.asarray(rows)
+        o_gpu = f64(out.cpu())[self.bsel][:, rows_idx][:, :, self.hsel]
+        l_gpu = lse.cpu().double().numpy()[self.bsel][:, self.hsel][:, :, rows_idx]
+        o_ref, l_ref = self.oracle.attend(self._slice(Q), self._slice(Kc), self._slice(Vc),
+                                          final, rows=rows_idx)
+        return o_gpu, o_ref, l_gpu, l_ref
+
+    def check_layout(self):
+        for tier in (NOISY, CLEAN):
+            got = self.gpu.layout(tier)
+            want = [-1 if s is None else s for s in self.oracle.model[tier].slots]
+            assert got == want, (tier, got, want)
+            assert self.gpu.chunk_count(tier) == self.oracle.model[tier].count

@@ -1,0 +1,103 @@
+"""The C ABI on the CPU: the library loads, exports what include/sa.h declares,
+validates configs, and its host-side cache plan matches the oracle bit for bit."""
+
+import ctypes
+
+import pytest
+import torch
+
+import block_causal_streaming_sa_b200 as sa
+from oracle.cache import RingCacheModel
+from sa_inputs import WORKLOADS
+
+
+def _cfg(**kw):
+    base = dict(batch=1, heads=2, head_dim=64, frames_per_chunk=3, tok_h=8, tok_w=8,
+                sink_chunks=1, window_chunks=2)
+    base.update(kw)
+    return sa.make_config(**base)
+
+
+def test_library_exports_every_declared_symbol():
+    syms = sa.header_symbols()
+    assert {"sa_create", "sa_append_chunk", "sa_attend", "sa_destroy"} <= set(syms)
+    handle = ctypes.CDLL(sa._binding.LIB_PATH)
+    for name in syms:
+        assert hasattr(handle, name), name
+    sa.lib()  # argtypes for every declared symbol bind
+    assert set(syms) <= set(sa._binding._SIGNATURES)
+
+
+def test_validate_config_and_required_bytes():
+    assert sa.sa_validate_config(_cfg()) == sa.SA_OK
+    assert sa.sa_validate_config(_cfg(head_dim=96)) == sa.SA_ERR_UNSUPPORTED
+    assert sa.sa_validate_config(_cfg(batch=0)) == sa.SA_ERR_INVALID_ARG
+    assert sa.sa_validate_config(_cfg(window_chunks=0)) == sa.SA_ERR_INVALID_ARG
+    assert sa.sa_validate_config(_cfg(sink_chunks=-1)) == sa.SA_ERR_INVALID_ARG
+    assert sa.sa_validate_config(_cfg(sink_chunks=8, window_chunks=9)) == sa.SA_ERR_UNSUPPORTED
+    assert sa.sa_validate_config(_cfg(softmax_scale=float("nan"))) == sa.SA_ERR_INVALID_ARG
+    assert sa.sa_required_bytes(_cfg(head_dim=96)) == 0
+    small = sa.sa_required_bytes(_cfg())
+    big = sa.sa_required_bytes(_cfg(window_chunks=5))
+    # two tiers x (S + W - 1) slots x (K + V) x B*H*L*D bf16 at least
+    L = 3 * 8 * 8
+    assert small >= 2 * 2 * 2 * (1 * 2 * L * 64) * 2
+    assert big - small >= 2 * 3 * 2 * (2 * L * 64) * 2
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_plan_matches_oracle_cache_model(name):
+    """ids, slots and relocated temporal bases of every chunk of the stream."""
+    w = WORKLOADS[name]
+    cfg = sa.make_config(**w.config_dict())
+    model = RingCacheModel(w.sink, w.window)
+    slot_of_id = {}
+    for c in range(max(w.stream, 40)):
+        ids, slots, tbase = sa.sa_plan(cfg, c)
+        assert ids == model.attended()
+        ranks = model.ranks()
+        assert tbase == [ranks[j] * w.frames for j in ids]
+        assert slots == [slot_of_id[j] if j != c else -1 for j in ids]
+        slot, _ = model.append()
+        assert sa.sa_slot_of(cfg, c) == (-1 if slot is None else slot)
+        slot_of_id[c] = slot
+
+
+@pytest.mark.parametrize("sink,window", [(0, 1), (0, 2), (2, 1), (3, 5), (7, 9), (0, 16)])
+def test_plan_degenerate_and_extreme_windows(sink, window):
+    cfg = _cfg(sink_chunks=sink, window_chunks=window)
+    model = RingCacheModel(sink, window)
+    for c in range(60):
+        ids, slots, tbase = sa.sa_plan(cfg, c)
+        assert ids == model.attended()
+        assert max(tbase) + 2 <= (sink + window) * 3 - 1
+        slot, _ = model.append()
+        assert sa.sa_slot_of(cfg, c) == (-1 if slot is None else slot)
+
+
+def test_plan_rejects_bad_arguments():
+    with pytest.raises(sa.SaError):
+        sa.sa_plan(_cfg(), -1)
+    with pytest.raises(sa.SaError):
+        sa.sa_plan(_cfg(head_dim=96), 0)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_create_without_gpu_fails_cleanly():
+    with pytest.raises(sa.SaError) as e:
+        sa.sa_create(_cfg(), 0x100000, 1 << 30)
+    assert e.value.status in (sa.SA_ERR_INVALID_ARG, sa.SA_ERR_CUDA)
+    with pytest.raises(sa.SaError):
+        sa.sa_create(_cfg(), 0, 1 << 30)
+    with pytest.raises(sa.SaError):
+        sa.sa_create(_cfg(), 0x100000, 16)
+
+
+def test_null_handle_calls_fail_cleanly():
+    lib = sa.lib()
+    assert lib.sa_attend(None, None, None, None, 0, None, None, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_append_chunk(None, 0, None, None, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_reset(None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_chunk_count(None, 0) < 0
+    assert lib.sa_destroy(None) == sa.SA_OK
+    assert sa.last_error() != ""
