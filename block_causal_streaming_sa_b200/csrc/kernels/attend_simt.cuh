@@ -1,13 +1,14 @@
 // Plain fp32 SIMT attention over the sink + window chunks: one warp per query
 // row, lanes split the head dimension, exact exp2f, online softmax over keys in
 // ascending chunk order. Reads the same cache layout as the tensor-core kernel
-// and applies the same query-side relocated rotation (rounded to bf16 like the
+// and applies the same query-side relocated rotation (rounded to fp16 like the
 // MMA operand), so it is an independent check of the tensor-core machinery.
 // Debug path only: sa_debug_attend_simt.
 #pragma once
 
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "../sa_internal.h"
 #include "rope.cuh"
@@ -44,8 +45,8 @@ __global__ void __launch_bounds__(256) attend_simt_kernel(AttendParams p) {
     for (int pp = 0; pp < DPL / 2; ++pp) {
       const float2 cs = rope_cs(p.rope, lane * (DPL / 2) + pp, grp.t_delta + f, y, x);
       const float a = qraw[2 * pp], bb = qraw[2 * pp + 1];
-      q[2 * pp] = __bfloat162float(__float2bfloat16_rn(fmaf(a, cs.x, -bb * cs.y)));
-      q[2 * pp + 1] = __bfloat162float(__float2bfloat16_rn(fmaf(a, cs.y, bb * cs.x)));
+      q[2 * pp] = __half2float(__float2half_rn(fmaf(a, cs.x, -bb * cs.y)));
+      q[2 * pp + 1] = __half2float(__float2half_rn(fmaf(a, cs.y, bb * cs.x)));
     }
     const __nv_bfloat16 *kb, *vb;
     size_t vstride;
@@ -63,7 +64,8 @@ __global__ void __launch_bounds__(256) attend_simt_kernel(AttendParams p) {
       const __nv_bfloat16* vr = vb + static_cast<size_t>(n) * vstride + lane * DPL;
       float s = 0.f;
 #pragma unroll
-      for (int d = 0; d < DPL; ++d) s = fmaf(q[d], __bfloat162float(kr[d]), s);
+      for (int d = 0; d < DPL; ++d)
+        s = fmaf(q[d], __half2float(reinterpret_cast<const __half*>(kr)[d]), s);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
       const float s2 = s * p.scale_log2;

@@ -58,8 +58,9 @@ struct TcShape {
   static constexpr int kTmemCols = 512;
   static constexpr int kDt = D - 4 * (D / 6);             // temporal band width
   static constexpr int kTChunks = (kDt + 7) / 8;           // 16-byte chunks holding it
-  static constexpr uint32_t kIdescQK = ptx::idesc_bf16_f32(BM, BN, 0);
-  static constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(BM, D, 1);
+  static constexpr uint32_t kIdescQK = ptx::idesc_f32acc(BM, BN, 0, 0);  // fp16 Q~, K~
+  static constexpr uint32_t kIdescPV = ptx::idesc_f32acc(BM, D, 1, 1);   // bf16 P, V
+
   __host__ __device__ static constexpr int col_s(int i) { return i * 128; }
   __host__ __device__ static constexpr int col_o(int i) { return 256 + i * D; }
   __host__ __device__ static constexpr int col_p(int i) { return i * 128 + 64; }  // bf16 P

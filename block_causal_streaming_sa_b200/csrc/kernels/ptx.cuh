@@ -213,13 +213,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
-// Instruction descriptor of kind::f16: bf16 A and B, fp32 accumulator,
-// M x N tile, A K-major, B K-major (b_mn_major = 0) or MN-major (1).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn_major) {
-  return (1u << 4)       // accumulator F32
-         | (1u << 7)     // A = BF16
-         | (1u << 10)    // B = BF16
-         | (0u << 15)    // A K-major
+// Instruction descriptor of kind::f16 with an fp32 accumulator: A and B both
+// fp16 (ab_bf16 = 0) or both bf16 (1), M x N tile, A K-major, B K-major
+// (b_mn_major = 0) or MN-major (1).
+__host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, int ab_bf16, int b_mn_major) {
+  return (1u << 4)                                    // accumulator F32
+         | (static_cast<uint32_t>(ab_bf16) << 7)      // A format: F16 = 0, BF16 = 1
+         | (static_cast<uint32_t>(ab_bf16) << 10)     // B format
+         | (0u << 15)                                 // A K-major
          | (static_cast<uint32_t>(b_mn_major) << 16) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
@@ -230,6 +231,13 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Round two floats to fp16 (nearest even, saturating at +-65504) and pack.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

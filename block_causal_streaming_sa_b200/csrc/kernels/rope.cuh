@@ -4,7 +4,7 @@
 // each token's position in space and in time) is applied with the band
 // reading [t | h | w], pair (2i, 2i+1) of a band turned by pos * theta^(-2i/d).
 //
-// Keys enter the cache rotated by their IN-CHUNK position (frame f within the
+// Keys enter the cache rotated by their IN-CHUNK position and stored as fp16 (frame f within the
 // chunk, row y, column x). The relocated temporal base of a cached chunk
 // ("RoPE relocation", section 选择三 of "Vidu S2 vs PixVerse R2") changes as the
 // window slides, so it is not baked in: a rotation by rank(j) * F of every key
@@ -33,12 +33,15 @@ __device__ __forceinline__ float2 rope_cs(const RopeTables& rt, int pair, int po
   return __ldg(&rt.w[x * rt.dw2 + pair]);
 }
 
+// Turn one bf16 pair by (cos, sin) in fp32; the result is rounded once to fp16,
+// the operand type of the score MMA (11 significant bits instead of bf16's 8).
 __device__ __forceinline__ uint32_t rope_pair(uint32_t ab, float2 cs) {
   const float a = bf16_lo(ab), b = bf16_hi(ab);
-  return ptx::pack_bf16x2(fmaf(a, cs.x, -b * cs.y), fmaf(a, cs.y, b * cs.x));
+  return ptx::pack_f16x2(fmaf(a, cs.x, -b * cs.y), fmaf(a, cs.y, b * cs.x));
 }
 
-// Rotate the 8 values (4 pairs) of 16-byte chunk `c` of a head vector.
+// Rotate the 8 bf16 values (4 pairs) of 16-byte chunk `c` of a head vector into
+// 8 fp16 values.
 __device__ __forceinline__ uint4 rope_chunk(uint4 v, int c, const RopeTables& rt, int pos_t, int y,
                                             int x) {
   v.x = rope_pair(v.x, rope_cs(rt, 4 * c + 0, pos_t, y, x));
@@ -63,7 +66,7 @@ __device__ __forceinline__ void st_v4(void* p, uint4 v) {
 }
 
 // One block per token (b, l); thread t moves 16-byte chunk t % (D/8) of head
-// t / (D/8). blockIdx.y: 0 = K (rotated), 1 = V (copied). Loads are fully
+// t / (D/8). blockIdx.y: 0 = K (bf16 in, rotated, fp16 out), 1 = V (bf16, copied). Loads are fully
 // coalesced (a token's H*D values are contiguous); each head's 2*D bytes are
 // stored contiguously into its [B, H, L, D] plane.
 __global__ void rope_transpose_kernel(AppendParams p) {

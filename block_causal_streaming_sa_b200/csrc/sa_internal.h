@@ -26,8 +26,8 @@ struct RopeTables {
 };
 
 // Rotate-and-transpose of one chunk: in [B, L, H, D] -> out [B, H, L, D].
-// K rows are turned by their in-chunk (frame, row, column) position; V rows
-// (blockIdx.y == 1) are copied.
+// K rows (bf16) are turned by their in-chunk (frame, row, column) position and
+// written as fp16; V rows (blockIdx.y == 1) are copied as bf16.
 struct AppendParams {
   const __nv_bfloat16* k_in;
   const __nv_bfloat16* v_in;  // may be null (K only)
@@ -49,8 +49,9 @@ struct AttendParams {
   const __nv_bfloat16* q;        // [B, L, H, D] unrotated
   __nv_bfloat16* o;              // [B, L, H, D]
   float* lse;                    // [B, H, L] or null
-  const __nv_bfloat16* cache;    // selected tier: [slot][K|V][B][H][L][D], K rotated in-chunk
-  const __nv_bfloat16* k_cur;    // current chunk K, rotated in-chunk: [B][H][L][D]
+  const __nv_bfloat16* cache;    // selected tier: [slot][K|V][B][H][L][D]; K planes hold
+                                 // fp16 keys rotated in-chunk, V planes bf16
+  const __nv_bfloat16* k_cur;    // current chunk K (fp16 bits), rotated in-chunk: [B][H][L][D]
   const __nv_bfloat16* v_cur;    // current chunk V as passed: [B][L][H][D]
   int B, L, H, D;
   int n_groups;

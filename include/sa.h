@@ -84,7 +84,7 @@ SA_API int sa_validate_config(const sa_config* cfg);
 
 /* Bytes of device memory sa_create needs for cfg (0 if cfg is invalid):
  * a status word, fp32 RoPE tables, both cache tiers ((S + W - 1) slots of K and
- * V each, layout [slot][K|V][B][H][L][D]) and one rotated-key chunk of scratch
+ * V each, layout [slot][K|V][B][H][L][D], K fp16, V bf16) and one rotated-key chunk of scratch
  * for the chunk being generated. Host only. */
 SA_API size_t sa_required_bytes(const sa_config* cfg);
 
@@ -108,7 +108,9 @@ SA_API int sa_reset(sa_handle* h);
  * window slot S + (n - S) mod (W - 1), overwriting (evicting) the oldest
  * non-sink chunk once the window is full; with W == 1 a non-sink chunk is not
  * stored. K is rotated by its in-chunk (frame, row, column) position on the way
- * in; the relocated temporal offset is applied at attend time.
+ * in and kept as fp16 (the score MMA's operand type; rotated pairs must keep a
+ * norm below 65504, larger ones saturate); V is kept as bf16. The relocated
+ * temporal offset is applied at attend time.
  * A tier may run at most one chunk ahead of the other: appending to the tier
  * that is already ahead is SA_ERR_STATE. K and V may be freed once the launch
  * on `stream` has run. */
@@ -123,7 +125,8 @@ SA_API int sa_append_chunk(sa_handle* h, int tier, const void* K, const void* V,
  * all bidirectional inside the chunk. Chunk j sits at temporal position
  * rank(j) * F + frame, rank = index of j among the attended chunks in
  * ascending id order, so positions stay below (S + W) * F.
- * Q, Kc, Vc: [B, L, H, D] bf16 (unrotated), read only.
+ * Q, Kc, Vc: [B, L, H, D] bf16 (unrotated), read only. Rotated Q and K enter
+ * the score MMA as fp16, P and V the output MMA as bf16; accumulation is fp32.
  * O: [B, L, H, D] bf16, fully overwritten (must not alias the inputs).
  * lse: optional [B, H, L] fp32 natural-log sum of exp of the scaled scores
  *      (NULL to skip), for merging partial attentions.

@@ -12,6 +12,25 @@ from oracle.stream import CLEAN, NOISY, OracleConfig, StreamOracle
 
 TOL = 1e-2  # max |O_gpu - O_oracle| on bf16 outputs with fp32 accumulation
 
+# O is returned in bf16, so rounding it alone moves an element by up to half an
+# ulp, 2^-8 |O| (8 significant bits). For |O| >= 2.56 that exceeds TOL by itself;
+# workloads whose outputs reach that size (the +-8 outlier stream) are held to
+# TOL beyond that unavoidable output rounding.
+HALF_ULP_BF16 = 2.0 ** -8
+
+
+def check_output(o_gpu, o_ref, what, allow_output_rounding=False):
+    """Assert the GPU output is within TOL of the oracle; returns (max err, excess)."""
+    d = np.abs(o_gpu - o_ref)
+    err = float(d.max())
+    excess = float((d - HALF_ULP_BF16 * np.abs(o_ref)).max())
+    if allow_output_rounding:
+        assert excess <= TOL, (f"{what}: max (|O - oracle| - half ulp of bf16 O) = {excess:.3e}"
+                               f" (plain max {err:.3e})")
+    else:
+        assert err <= TOL, f"{what}: max |O - oracle| = {err:.3e}"
+    return err, excess
+
 
 def f64(t):
     return t.to(torch.float64).numpy()

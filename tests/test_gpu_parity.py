@@ -5,16 +5,15 @@ import pytest
 import torch
 
 import block_causal_streaming_sa_b200 as sa
-from harness import TOL, Pair, f64, sample_rows
+from harness import TOL, Pair, check_output, f64, sample_rows
 from oracle.stream import CLEAN, NOISY
 from sa_inputs import WORKLOADS, Workload
 
 pytestmark = pytest.mark.gpu
 
 
-def _assert_close(o_gpu, o_ref, l_gpu, l_ref, what):
-    err = np.abs(o_gpu - o_ref).max()
-    assert err <= TOL, f"{what}: max |O - oracle| = {err:.3e}"
+def _assert_close(o_gpu, o_ref, l_gpu, l_ref, what, allow_output_rounding=False):
+    err, _ = check_output(o_gpu, o_ref, what, allow_output_rounding)
     lerr = np.abs(l_gpu - l_ref).max()
     assert lerr <= 1e-2, f"{what}: max |lse - oracle| = {lerr:.3e}"
     return err
@@ -151,14 +150,15 @@ def test_full_size_sampled_rows(case):
     step, on >= 256 sampled query rows per checked (b, h)."""
     name, heads, batches, nrows = case
     w = WORKLOADS[name]
+    big = w.outlier_frac > 0  # +-8 outliers in V: |O| reaches 4..8
     pair = Pair(w, batches=batches, heads=heads)
     rows = sample_rows(w.chunk_len, nrows, seed=7)
-    _assert_close(*pair.attend(0, w.steps == 1, rows=rows), f"{name} chunk 0")
+    _assert_close(*pair.attend(0, w.steps == 1, rows=rows), f"{name} chunk 0", big)
     first_evicting = w.sink + w.window  # this chunk's plan no longer holds chunk S
     while pair.chunk < first_evicting:
         pair.append()
     pair.check_layout()
     if w.steps > 1:
-        _assert_close(*pair.attend(0, False, rows=rows), f"{name} noisy step")
-    _assert_close(*pair.attend(w.steps - 1, True, rows=rows), f"{name} clean step")
+        _assert_close(*pair.attend(0, False, rows=rows), f"{name} noisy step", big)
+    _assert_close(*pair.attend(w.steps - 1, True, rows=rows), f"{name} clean step", big)
     assert pair.gpu.status() == sa.SA_OK
