@@ -23,6 +23,7 @@ SA_ERR_TIMEOUT = 5
 SA_TIER_NOISY = 0
 SA_TIER_CLEAN = 1
 SA_MAX_ATTENDED = 16
+SA_NOALLOC_MAX_KEY_BYTES = 64 << 20
 
 
 class SaConfig(ctypes.Structure):
@@ -63,6 +64,7 @@ _SIGNATURES = {
     "sa_stage_keys": (_I, [_P, _P, _P]),
     "sa_attend_staged": (_I, [_P, _P, _P, _I, _P, _P, _P]),
     "sa_debug_attend_simt": (_I, [_P, _P, _P, _P, _I, _P, _P, _P]),
+    "sa_attend_noalloc": (_I, [_P, _P, _P, _P, _I, _P, _P, _P]),
     "sa_chunk_count": (_I, [_P, _I]),
     "sa_debug_layout": (_I, [_P, _I, _I32P, _I]),
     "sa_plan": (_I, [_CFGP, ctypes.c_int32, _I32P, _I32P, _I32P, _I]),
@@ -157,6 +159,13 @@ def sa_attend_staged(handle, Q, Vc, step_is_final, O, lse=0, stream=0):
 def sa_debug_attend_simt(handle, Q, Kc, Vc, step_is_final, O, lse=0, stream=0):
     _check(lib().sa_debug_attend_simt(handle, _P(Q), _P(Kc), _P(Vc), int(bool(step_is_final)),
                                       _P(O), _P(lse or None), _P(stream)), handle)
+
+
+def sa_attend_noalloc(handle, Q, Kc, Vc, step_is_final, O, lse=0, stream=0):
+    """sa_attend that allocates nothing: its key scratch is a fixed array inside
+    the library (for callers that cannot allocate device memory)."""
+    _check(lib().sa_attend_noalloc(handle, _P(Q), _P(Kc), _P(Vc), int(bool(step_is_final)),
+                                   _P(O), _P(lse or None), _P(stream)), handle)
 
 
 def sa_chunk_count(handle, tier):

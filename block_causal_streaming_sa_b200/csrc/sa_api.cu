@@ -357,6 +357,109 @@ int attend_common(sa_handle* h, const void* Q, const void* Kc, const void* Vc, i
   return attend_staged(h, Q, Vc, step_is_final, O, lse, stream, simt);
 }
 
+// ---------------------------------------------------------------- sa_attend_noalloc
+// Key scratch of sa_attend_noalloc: a fixed device array instead of the
+// handle's region. In host code `g_noalloc_keys` names a host-side stand-in,
+// not a device address: the address is looked up once per device with
+// cudaGetSymbolAddress while that device is current.
+static __device__ __align__(256) uint8_t g_noalloc_keys[SA_NOALLOC_MAX_KEY_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+int noalloc_scratch(sa_handle* h, void** out) {
+  if (h->device < 0 || h->device >= kMaxDevices)
+    return h->fail(SA_ERR_UNSUPPORTED, "device ordinal too large for sa_attend_noalloc");
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[h->device] == nullptr) {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_keys);
+    if (e != cudaSuccess || ptr == nullptr)
+      return h->fail(SA_ERR_CUDA, std::string("cudaGetSymbolAddress of the static key scratch: ") +
+                                      cudaGetErrorString(e));
+    g_noalloc_addr[h->device] = ptr;
+  }
+  *out = g_noalloc_addr[h->device];
+  return SA_OK;
+}
+
+int attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc, int step_is_final,
+                   void* O, float* lse, sa_stream stream) {
+  int rc = check_handle(h);
+  if (rc != SA_OK) return rc;
+  if (Q == nullptr || Kc == nullptr || Vc == nullptr || O == nullptr)
+    return h->fail(SA_ERR_INVALID_ARG, "Q, Kc, Vc and O must be non-NULL");
+  if (!aligned16(Q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(O) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 || O == Q || O == Kc || O == Vc)
+    return h->fail(SA_ERR_INVALID_ARG, "Q, Kc, Vc, O must be 16-byte aligned, lse 4-byte "
+                                       "aligned, O must not alias an input");
+  if (h->count[0] != h->count[1])
+    return h->fail(SA_ERR_STATE, "both tiers must hold the same chunks before attending");
+  const Derived& d = h->d;
+  if (d.chunk_elems * sizeof(__nv_bfloat16) > SA_NOALLOC_MAX_KEY_BYTES)
+    return h->fail(SA_ERR_UNSUPPORTED,
+                   "B*H*L*D*2 bytes exceed SA_NOALLOC_MAX_KEY_BYTES (64 MiB) of sa_attend_noalloc");
+  rc = check_device(h);
+  if (rc != SA_OK) return rc;
+  void* scratch = nullptr;
+  rc = noalloc_scratch(h, &scratch);
+  if (rc != SA_OK) return rc;
+  __nv_bfloat16* keys = static_cast<__nv_bfloat16*>(scratch);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int tier = step_is_final ? SA_TIER_CLEAN : SA_TIER_NOISY;
+  const int c = h->count[0];
+
+  CUtensorMap tm_keys, tm_v;
+  if (!encode_planes(&tm_keys, keys, d, 1LL * d.B * d.H) || !encode_blhd(&tm_v, Vc, d))
+    return h->fail(SA_ERR_CUDA, "TMA descriptors for sa_attend_noalloc failed");
+
+  AttendParams ap;
+  std::memset(&ap, 0, sizeof(ap));
+  ap.q = static_cast<const __nv_bfloat16*>(Q);
+  ap.o = static_cast<__nv_bfloat16*>(O);
+  ap.lse = lse;
+  ap.cache = h->tier_base(tier);
+  ap.k_cur = keys;
+  ap.v_cur = static_cast<const __nv_bfloat16*>(Vc);
+  ap.B = d.B;
+  ap.L = d.L;
+  ap.H = d.H;
+  ap.D = d.D;
+  int ids[SA_MAX_ATTENDED];
+  const int n = plan_ids(d, c, ids);
+  ap.n_groups = n;
+  for (int g = 0; g < n; ++g) {
+    AttendGroup& grp = ap.groups[g];
+    grp.src = ids[g] == c ? 1 : 0;
+    grp.slot = ids[g] == c ? 0 : slot_of(d, ids[g]);
+    grp.t_delta = (n - 1 - g) * d.F;
+    grp.len = d.L;
+  }
+  ap.scale_log2 = d.scale * 1.4426950408889634f;
+  ap.rope = h->rope();
+  ap.status = h->status();
+
+  // Every element of the scratch that the attention reads is written first by
+  // this launch, so nothing has to start at zero.
+  rc = launch_rope_transpose(h, Kc, nullptr, keys, nullptr, s);
+  if (rc != SA_OK) return rc;
+  const CUtensorMap& tm_cache = h->has_cache ? h->tm_tier[tier] : tm_keys;
+  const int n_qt = (d.L + 127) / 128;
+  const long long n_work = 1LL * d.B * d.H * ((n_qt + 1) / 2);
+  const unsigned grid = static_cast<unsigned>(n_work < h->sm_count ? n_work : h->sm_count);
+  if (d.D == 128)
+    sa::attend_tc_kernel<128><<<grid, sa::TcShape<128>::kThreads, sa::TcShape<128>::kSmemBytes,
+                                s>>>(tm_cache, tm_keys, tm_v, ap);
+  else
+    sa::attend_tc_kernel<64><<<grid, sa::TcShape<64>::kThreads, sa::TcShape<64>::kSmemBytes,
+                               s>>>(tm_cache, tm_keys, tm_v, ap);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return h->fail(SA_ERR_CUDA, std::string("attend launch: ") + cudaGetErrorString(e));
+  return SA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -543,6 +646,11 @@ SA_API int sa_attend_staged(sa_handle* h, const void* Q, const void* Vc, int ste
 SA_API int sa_debug_attend_simt(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
                                 int step_is_final, void* O, float* lse, sa_stream stream) {
   return attend_common(h, Q, Kc, Vc, step_is_final, O, lse, stream, true);
+}
+
+SA_API int sa_attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
+                             int step_is_final, void* O, float* lse, sa_stream stream) {
+  return attend_noalloc(h, Q, Kc, Vc, step_is_final, O, lse, stream);
 }
 
 SA_API int sa_chunk_count(const sa_handle* h, int tier) {

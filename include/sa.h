@@ -147,6 +147,29 @@ SA_API int sa_stage_keys(sa_handle* h, const void* Kc, sa_stream stream);
 SA_API int sa_attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final,
                             void* O, float* lse, sa_stream stream);
 
+/* sa_attend for callers that cannot allocate device memory. (The pages have no
+ * counterpart to this call; it exists for integration.)
+ * Some callers may not call cudaMalloc at all: code running inside another
+ * framework's allocator-free region, a real-time loop that must not allocate
+ * after start-up, or a plugin that is handed only the tensors it works on.
+ * This call computes exactly what sa_attend computes, with the same arguments,
+ * but it allocates nothing and does not use the handle's key scratch: the
+ * generating chunk's rotated keys go to a fixed array of
+ * SA_NOALLOC_MAX_KEY_BYTES (64 MiB) compiled into the library. Every device
+ * that loads the library holds that array until the process exits.
+ * Limits and rules:
+ *  - B * H * L * D * 2 bytes must fit in SA_NOALLOC_MAX_KEY_BYTES, else
+ *    SA_ERR_UNSUPPORTED and nothing is launched;
+ *  - the array is shared by every call in the process on that device and keeps
+ *    the last call's keys: calls that overlap on the GPU (two streams, two
+ *    handles) race; order them (one stream, or events);
+ *  - the first call on a device looks up the array's device address (a
+ *    runtime symbol query); make that first call before any stream capture.
+ * Returns the same statuses as sa_attend. */
+#define SA_NOALLOC_MAX_KEY_BYTES (64u << 20)
+SA_API int sa_attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
+                             int step_is_final, void* O, float* lse, sa_stream stream);
+
 /* Same contract as sa_attend, computed by a plain fp32 SIMT kernel (one warp
  * per query row, no tensor cores). A debugging cross-check of the tensor-core
  * kernel, an order of magnitude slower; not used by sa_attend. */
