@@ -17,11 +17,16 @@
 //    P_i read from TMEM, written over the upper half of S_i, V MN-major in shared memory);
 //    the two query tiles ping-pong so one tile's softmax overlaps the other's
 //    MMAs;
-//  * warps 2-5 / 6-9: one warpgroup per query tile, thread = query row =
+//  * warps 4-7 / 8-11: one warpgroup per query tile, thread = query row =
 //    TMEM lane. Each writes its rotated query tile into shared memory, runs the
-//    online softmax on S rows read from TMEM (no cross-thread reduction: a
-//    thread owns a whole row), writes P back as bf16, rescales O in TMEM only
-//    when the running max grows by more than 2^8, and runs the epilogue;
+//    online softmax on S rows read from TMEM in one round trip (no cross-thread
+//    reduction: a thread owns a whole row; max and sum as 8-way trees), writes P
+//    back as bf16, rescales O in TMEM only when the running max grows by more
+//    than 2^8, and runs the epilogue;
+//  * registers: launched at 168 per thread (384 threads), warpgroup 0 (warps
+//    0-3: producer, MMA issuer, two idle) gives registers back with setmaxnreg
+//    (104) and the softmax warpgroups take them (200), so a whole 128-score row
+//    stays in registers without spills;
 //  * RoPE: keys are stored rotated by their in-chunk position; the relocated
 //    temporal base rank(j) * F of the attended chunk is applied by re-turning
 //    the temporal band of the query tile when the key stream moves to the next
@@ -48,13 +53,23 @@ struct TcShape {
   static constexpr int kTile = BM * D * 2;       // bytes of a Q, K or V tile (BM == BN)
   static constexpr int kBox = BN * 128;          // bytes of one 64-column TMA box
   static constexpr int NSTAGE = (D == 128) ? 4 : 8;
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 384;
+  // Register split (setmaxnreg): launched at kLaunchRegs per thread (the
+  // __launch_bounds__(384, 1) budget); warpgroup 0 (producer, MMA) drops to
+  // kRegsCtl, the two softmax warpgroups rise to kRegsSoftmax.
+  // 128 * 56 + 256 * 224 = 64512 = 384 * 168 (the launch pool), and per SM
+  // sub-partition 56 + 224 + 224 = 504 <= 512 registers per thread slot.
+  static constexpr int kLaunchRegs = 168;
+  static constexpr int kRegsCtl = 104;
+  static constexpr int kRegsSoftmax = 200;
+  static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= kThreads * kLaunchRegs, "register split");
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kTile;
   static constexpr int kOffQRaw = kOffKV + NSTAGE * kTile;  // raw temporal chunks of both Q tiles
   static constexpr int kQRawRow = ((D - 4 * (D / 6) + 7) / 8) * 16;
   static constexpr int kOffBar = kOffQRaw + 2 * BM * kQRawRow;
-  static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + barrier area + alignment slack
+  static constexpr int kOffGroups = kOffBar + 256;          // attended-chunk table
+  static constexpr int kSmemBytes = kOffGroups + 256 + 1024;  // + table + alignment slack
   static constexpr int kTmemCols = 512;
   static constexpr int kDt = D - 4 * (D / 6);             // temporal band width
   static constexpr int kTChunks = (kDt + 7) / 8;           // 16-byte chunks holding it
@@ -98,7 +113,7 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tm_cache,
                      const __grid_constant__ CUtensorMap tm_kcur,
                      const __grid_constant__ CUtensorMap tm_vcur,
@@ -115,6 +130,14 @@ __global__ void __launch_bounds__(320, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // The attended-chunk table, indexed by a runtime chunk counter, lives in shared
+  // memory (dynamic indexing of a kernel parameter would copy it to local memory).
+  AttendGroup* groups = reinterpret_cast<AttendGroup*>(smem + T::kOffGroups);
+  static_assert(sizeof(AttendGroup) * kMaxGroups <= 256, "group table");
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int g = 0; g < kMaxGroups; ++g) groups[g] = p.groups[g];
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < T::NSTAGE; ++s) {
@@ -144,8 +167,10 @@ __global__ void __launch_bounds__(320, 1)
   const int n_pairs = (n_qt + 1) / 2;
   const int n_work = p.B * p.H * n_pairs;
   int n_kt_total = 0;
-  for (int g = 0; g < p.n_groups; ++g) n_kt_total += (p.groups[g].len + T::BN - 1) / T::BN;
+  for (int g = 0; g < p.n_groups; ++g) n_kt_total += (groups[g].len + T::BN - 1) / T::BN;
 
+  if (warp < 4) {
+  ptx::setmaxnreg_dec<T::kRegsCtl>();
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -159,7 +184,7 @@ __global__ void __launch_bounds__(320, 1)
         const int bh = w / n_pairs;
         const int b = bh / p.H, h = bh - b * p.H;
         for (int g = 0; ok && g < p.n_groups; ++g) {
-          const AttendGroup grp = p.groups[g];
+          const AttendGroup grp = groups[g];
           const int nkt = (grp.len + T::BN - 1) / T::BN;
           for (int t = 0; ok && t < nkt; ++t) {
             for (int kv = 0; kv < 2; ++kv) {
@@ -278,9 +303,11 @@ __global__ void __launch_bounds__(320, 1)
       ptx::umma_commit(bar(T::DRAIN()));
       ptx::mbar_wait(bar(T::DRAIN()), 0, &no_abort, p.status);
     }
+  }
   } else {
+    ptx::setmaxnreg_inc<T::kRegsSoftmax>();
     // ------------------------------------------------------------ softmax warpgroups
-    const int i = (warp - 2) >> 2;  // query tile of this warpgroup
+    const int i = (warp - 4) >> 2;  // query tile of this warpgroup
     const int quarter = warp & 3;   // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;
     const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
@@ -306,7 +333,7 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t q_raw = sbase + T::kOffQRaw + (i * T::BM + r) * T::kQRawRow;
       {
         const uint4* src = reinterpret_cast<const uint4*>(p.q + row_off);
-        const int td0 = p.groups[0].t_delta;
+        const int td0 = groups[0].t_delta;
 #pragma unroll 2
         for (int c = 0; c < D / 8; ++c) {
           uint4 v = valid ? ld_nc_v4(src + c) : make_uint4(0u, 0u, 0u, 0u);
@@ -320,7 +347,7 @@ __global__ void __launch_bounds__(320, 1)
       float m = -INFINITY, lsum = 0.f;
       int kt = 0;
       for (int g = 0; ok && g < p.n_groups; ++g) {
-        const int len = p.groups[g].len;
+        const int len = groups[g].len;
         const int nkt = (len + T::BN - 1) / T::BN;
         for (int t = 0; t < nkt; ++t, ++kt) {
           if (!ptx::mbar_wait(bar(T::SFULL(i)), s_phase, abort_flag, p.status)) {
@@ -329,33 +356,30 @@ __global__ void __launch_bounds__(320, 1)
           }
           s_phase ^= 1u;
           ptx::tc_fence_after();
-          // Scores of keys [col0, col0 + 64) of this row, keys past the chunk end masked.
+          // The whole score row (128 fp32) in one round trip; keys past the chunk end masked.
           const int nvalid = min(T::BN, len - t * T::BN);
-          uint32_t sr[2][32];
-          auto load_half = [&](int col0) {
-            ptx::tmem_ld32(tS + col0, sr[0]);
-            ptx::tmem_ld32(tS + col0 + 32, sr[1]);
-            ptx::tmem_wait_ld();
-            if (nvalid < col0 + 64) {
+          uint32_t sr[4][32];
 #pragma unroll
-              for (int j = 0; j < 2; ++j)
+          for (int j = 0; j < 4; ++j) ptx::tmem_ld32(tS + j * 32, sr[j]);
+          ptx::tmem_wait_ld();
+          if (nvalid < T::BN) {
 #pragma unroll
-                for (int c = 0; c < 32; ++c)
-                  if (col0 + j * 32 + c >= nvalid) sr[j][c] = __float_as_uint(-INFINITY);
-            }
-          };
-          auto half_max = [&]() {
-            float mx = -INFINITY;
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
+              for (int c = 0; c < 32; ++c)
+                if (j * 32 + c >= nvalid) sr[j][c] = __float_as_uint(-INFINITY);
+          }
+          // Row max as a tree over 8 independent running maxima.
+          float mx8[8];
 #pragma unroll
-              for (int c = 0; c < 32; ++c) mx = fmaxf(mx, __uint_as_float(sr[j][c]));
-            return mx;
-          };
-          load_half(0);
-          float mx = half_max();
-          load_half(64);
-          mx = fmaxf(mx, half_max());
+          for (int a = 0; a < 8; ++a) mx8[a] = __uint_as_float(sr[0][a]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (j > 0 || c >= 8) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[j][c]));
+          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
           const float m_new = fmaxf(m, mx * p.scale_log2);
           const bool need = m_new > m + 8.0f;
           float alpha = 1.f;
@@ -364,29 +388,25 @@ __global__ void __launch_bounds__(320, 1)
             m = m_new;
           }
           // P = 2^(s * scale * log2 e - m) as bf16 pairs in columns 64..127 of the S
-          // region (P of key k in column 64 + k / 2). Keys 64..127 first, from the
-          // registers: their P overwrites scores of keys 96..127, already read. Then
-          // keys 0..63 after reloading them: their P overwrites keys 64..95, also read.
-          float rs = 0.f;
-          auto exp_store = [&](int pcol) {
+          // region (P of key k in column 64 + k / 2); the sum over 8 partial sums.
+          float rs8[8];
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              uint32_t pk[16];
+          for (int a = 0; a < 8; ++a) rs8[a] = 0.f;
 #pragma unroll
-              for (int c = 0; c < 16; ++c) {
-                const float p0 =
-                    ptx::ex2(fmaf(__uint_as_float(sr[j][2 * c]), p.scale_log2, -m));
-                const float p1 =
-                    ptx::ex2(fmaf(__uint_as_float(sr[j][2 * c + 1]), p.scale_log2, -m));
-                rs += p0 + p1;
-                pk[c] = ptx::pack_bf16x2(p0, p1);
-              }
-              ptx::tmem_st16(tS + pcol + j * 16, pk);
+          for (int j = 0; j < 4; ++j) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const float p0 = ptx::ex2(fmaf(__uint_as_float(sr[j][2 * c]), p.scale_log2, -m));
+              const float p1 =
+                  ptx::ex2(fmaf(__uint_as_float(sr[j][2 * c + 1]), p.scale_log2, -m));
+              rs8[c & 7] += p0 + p1;
+              pk[c] = ptx::pack_bf16x2(p0, p1);
             }
-          };
-          exp_store(96);
-          load_half(0);
-          exp_store(64);
+            ptx::tmem_st16(tS + 64 + j * 16, pk);
+          }
+          const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) +
+                           ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
           lsum = lsum * alpha + rs;
           if (__any_sync(0xffffffffu, need && kt > 0)) {
 #pragma unroll
@@ -400,7 +420,7 @@ __global__ void __launch_bounds__(320, 1)
             }
           }
           if (t == nkt - 1 && g + 1 < p.n_groups) {
-            const int td = p.groups[g + 1].t_delta;
+            const int td = groups[g + 1].t_delta;
 #pragma unroll 2
             for (int c = 0; c < T::kTChunks; ++c)
               st_shared_v4(q_smem + sw128_offset(r, c),

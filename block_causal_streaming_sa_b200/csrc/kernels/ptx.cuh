@@ -225,6 +225,18 @@ __host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, int ab_bf16, i
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// ---------------------------------------------------------------- register split
+
+// Whole warpgroup: lower / raise this warp's register budget (multiple of 8).
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- misc
 
 __device__ __forceinline__ float ex2(float x) {

@@ -567,6 +567,17 @@ SA_API int sa_create(const sa_config* cfg, void* dev_buf, size_t bytes, sa_handl
     delete h;
     return SA_ERR_CUDA;
   }
+  // The kernel's register split assumes it is launched with exactly
+  // TcShape::kLaunchRegs registers per thread; refuse to run otherwise.
+  cudaFuncAttributes fa128, fa64;
+  if (cudaFuncGetAttributes(&fa128, sa::attend_tc_kernel<128>) != cudaSuccess ||
+      cudaFuncGetAttributes(&fa64, sa::attend_tc_kernel<64>) != cudaSuccess ||
+      fa128.numRegs != sa::TcShape<128>::kLaunchRegs ||
+      fa64.numRegs != sa::TcShape<64>::kLaunchRegs) {
+    g_error = "attention kernel built with an unexpected register count";
+    delete h;
+    return SA_ERR_UNSUPPORTED;
+  }
   cudaError_t e = cudaFuncSetAttribute(sa::attend_tc_kernel<128>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        sa::TcShape<128>::kSmemBytes);
