@@ -279,43 +279,52 @@ def run_ours(args, w):
     out = torch.empty(w.shape(), dtype=torch.bfloat16, device=dev)
     out_host = torch.empty(w.shape(), dtype=torch.bfloat16).pin_memory()
 
-    attn = sa.StreamingAttention(w.config_dict(), device=dev)
-    h = attn.handle
+    # One handle (its own two-tier cache) per attention layer of the workload.
+    layers = [sa.StreamingAttention(w.config_dict(), device=dev) for _ in range(w.layers)]
+    attn = layers[0]
     sp = stream.cuda_stream
     flops = attend_flops(w)
     steps_per_chunk = w.steps
-    appends_per_chunk = 2
+    attends_per_chunk = steps_per_chunk * w.layers
+    appends_per_chunk = 2 * w.layers
+
+    def append_all(s):
+        for layer in layers:
+            h = layer.handle
+            sa.sa_append_chunk(h, sa.SA_TIER_NOISY, s["Kn"].data_ptr(), s["Vn"].data_ptr(), sp)
+            sa.sa_append_chunk(h, sa.SA_TIER_CLEAN, s["Kcl"].data_ptr(), s["Vcl"].data_ptr(), sp)
 
     def chunk_step(s, ev=None):
-        """One chunk: every denoising step's attention, then the two appends."""
+        """One chunk: every denoising step's attention in every layer, then the appends."""
+        a = 0
         for k in range(steps_per_chunk):
             final = k == steps_per_chunk - 1
-            sa.sa_stage_keys(h, s["Kc"].data_ptr(), sp)
-            if ev is not None:
-                ev[0][k].record(stream)
-            sa.sa_attend_staged(h, s["Q"].data_ptr(), s["Vc"].data_ptr(), final, out.data_ptr(),
-                                0, sp)
-            if ev is not None:
-                ev[1][k].record(stream)
+            for layer in layers:
+                h = layer.handle
+                sa.sa_stage_keys(h, s["Kc"].data_ptr(), sp)
+                if ev is not None:
+                    ev[0][a].record(stream)
+                sa.sa_attend_staged(h, s["Q"].data_ptr(), s["Vc"].data_ptr(), final,
+                                    out.data_ptr(), 0, sp)
+                if ev is not None:
+                    ev[1][a].record(stream)
+                a += 1
         if ev is not None:
             ev[2].record(stream)
-        sa.sa_append_chunk(h, sa.SA_TIER_NOISY, s["Kn"].data_ptr(), s["Vn"].data_ptr(), sp)
-        sa.sa_append_chunk(h, sa.SA_TIER_CLEAN, s["Kcl"].data_ptr(), s["Vcl"].data_ptr(), sp)
+        append_all(s)
         if ev is not None:
             ev[3].record(stream)
 
     with torch.cuda.stream(stream):
         # Fill the window so every timed chunk attends to S + W chunks.
         for c in range(w.sink + w.window - 1):
-            s = pool[c % 2]
-            sa.sa_append_chunk(h, sa.SA_TIER_NOISY, s["Kn"].data_ptr(), s["Vn"].data_ptr(), sp)
-            sa.sa_append_chunk(h, sa.SA_TIER_CLEAN, s["Kcl"].data_ptr(), s["Vcl"].data_ptr(), sp)
+            append_all(pool[c % 2])
         for i in range(args.warmup):
             chunk_step(pool[i % 2])
         stream.synchronize()
 
         mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-        evs = [([mk() for _ in range(steps_per_chunk)], [mk() for _ in range(steps_per_chunk)],
+        evs = [([mk() for _ in range(attends_per_chunk)], [mk() for _ in range(attends_per_chunk)],
                 mk(), mk()) for _ in range(args.steps)]
         start, stop = mk(), mk()
         barrier()
@@ -330,7 +339,7 @@ def run_ours(args, w):
         clock_info = clocks.stop() if clocks is not None else None
         barrier()
         ms_local = start.elapsed_time(stop)
-        attend_ms = [e[0][k].elapsed_time(e[1][k]) for e in evs for k in range(steps_per_chunk)]
+        attend_ms = [e[0][k].elapsed_time(e[1][k]) for e in evs for k in range(attends_per_chunk)]
         append_ms = [e[2].elapsed_time(e[3]) for e in evs]
         assert attn.status(stream) == sa.SA_OK, "device status word reports a timeout"
 
@@ -361,9 +370,9 @@ def run_ours(args, w):
 
     ms_max = max_over_ranks(ms_local)
     e2e_ms_max = max_over_ranks(e2e_ms_local)
-    total_flops = flops * steps_per_chunk * args.steps * world
+    total_flops = flops * attends_per_chunk * args.steps * world
     value = total_flops / (ms_max * 1e-3) / 1e12
-    e2e_value = flops * steps_per_chunk * e2e_steps * world / (e2e_ms_max * 1e-3) / 1e12
+    e2e_value = flops * attends_per_chunk * e2e_steps * world / (e2e_ms_max * 1e-3) / 1e12
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -380,6 +389,7 @@ def run_ours(args, w):
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     append_bytes = appends_per_chunk * 2 * 2 * (w.batch * w.chunk_len * w.heads * w.head_dim * 2)
+    # (per append of one tier: K and V, each read once and written once)
     append_gbs = append_bytes / (statistics.fmean(append_ms) * 1e-3) / 1e9
     cache_bytes_read = 2 * (w.kv_len - w.chunk_len) * w.batch * w.heads * w.head_dim * 2
     line = {
@@ -398,8 +408,8 @@ def run_ours(args, w):
         "config": {
             "workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
             "chunk_tokens": w.chunk_len, "kv_tokens": w.kv_len, "sink_chunks": w.sink,
-            "window_chunks": w.window, "denoise_steps_per_chunk": w.steps,
-            "step": "all denoising attentions of one chunk + noisy and clean append",
+            "window_chunks": w.window, "denoise_steps_per_chunk": w.steps, "layers": w.layers,
+            "step": "all denoising attentions of one chunk (every layer) + noisy and clean appends",
             "l2": f"inputs larger than L2: {cache_bytes_read / 2**20:.0f} MiB of cached K/V "
                   f"read per attention vs {L2_BYTES / 2**20:.0f} MiB L2",
             "parallelism": f"replicas{world}" if world > 1 else "single",
@@ -417,7 +427,7 @@ def run_ours(args, w):
         "attention_tflops_kernel": achieved,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms_max / e2e_steps},
-        "gpu_launches": args.steps * (2 * steps_per_chunk + appends_per_chunk),
+        "gpu_launches": args.steps * (2 * attends_per_chunk + appends_per_chunk),
         "clocks": clock_info,
         "cpu_baseline": cpu,
     }

@@ -65,6 +65,7 @@ _SIGNATURES = {
     "sa_attend_staged": (_I, [_P, _P, _P, _I, _P, _P, _P]),
     "sa_debug_attend_simt": (_I, [_P, _P, _P, _P, _I, _P, _P, _P]),
     "sa_attend_noalloc": (_I, [_P, _P, _P, _P, _I, _P, _P, _P]),
+    "sa_debug_exp2": (_I, [_I, _P, _P, _I, _P]),
     "sa_chunk_count": (_I, [_P, _I]),
     "sa_debug_layout": (_I, [_P, _I, _I32P, _I]),
     "sa_plan": (_I, [_CFGP, ctypes.c_int32, _I32P, _I32P, _I32P, _I]),
@@ -166,6 +167,10 @@ def sa_attend_noalloc(handle, Q, Kc, Vc, step_is_final, O, lse=0, stream=0):
     the library (for callers that cannot allocate device memory)."""
     _check(lib().sa_attend_noalloc(handle, _P(Q), _P(Kc), _P(Vc), int(bool(step_is_final)),
                                    _P(O), _P(lse or None), _P(stream)), handle)
+
+
+def sa_debug_exp2(use_polynomial, x, y, n, stream=0):
+    _check(lib().sa_debug_exp2(int(bool(use_polynomial)), _P(x), _P(y), int(n), _P(stream)))
 
 
 def sa_chunk_count(handle, tier):

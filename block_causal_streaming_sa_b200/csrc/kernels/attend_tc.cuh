@@ -20,7 +20,9 @@
 //  * warps 4-7 / 8-11: one warpgroup per query tile, thread = query row =
 //    TMEM lane. Each writes its rotated query tile into shared memory, runs the
 //    online softmax on S rows read from TMEM in one round trip (no cross-thread
-//    reduction: a thread owns a whole row; max and sum as 8-way trees), writes P
+//    reduction: a thread owns a whole row; max as an 8-way tree of 3-input
+//    maxima, scale-and-subtract and the row sum in packed fp32x2 instructions,
+//    1 exponential in 8 on the FMA pipe by a fitted polynomial), writes P
 //    back as bf16, rescales O in TMEM only when the running max grows by more
 //    than 2^8, and runs the epilogue;
 //  * registers: launched at 168 per thread (384 threads), warpgroup 0 (warps
@@ -369,17 +371,19 @@ __global__ void __launch_bounds__(384, 1)
               for (int c = 0; c < 32; ++c)
                 if (j * 32 + c >= nvalid) sr[j][c] = __float_as_uint(-INFINITY);
           }
-          // Row max as a tree over 8 independent running maxima.
+          // Row max as a tree over 8 independent running maxima (3-input max).
           float mx8[8];
 #pragma unroll
           for (int a = 0; a < 8; ++a) mx8[a] = __uint_as_float(sr[0][a]);
 #pragma unroll
           for (int j = 0; j < 4; ++j)
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (j > 0 || c >= 8) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[j][c]));
-          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            for (int c = 0; c < 32; c += 2)
+              if (j > 0 || c >= 8)
+                mx8[(c >> 1) & 7] = ptx::fmax3(mx8[(c >> 1) & 7], __uint_as_float(sr[j][c]),
+                                               __uint_as_float(sr[j][c + 1]));
+          const float mx = fmaxf(ptx::fmax3(mx8[0], mx8[1], mx8[2]),
+                                 fmaxf(ptx::fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
           const float m_new = fmaxf(m, mx * p.scale_log2);
           const bool need = m_new > m + 8.0f;
           float alpha = 1.f;
@@ -389,24 +393,33 @@ __global__ void __launch_bounds__(384, 1)
           }
           // P = 2^(s * scale * log2 e - m) as bf16 pairs in columns 64..127 of the S
           // region (P of key k in column 64 + k / 2); the sum over 8 partial sums.
+          // x = s * scale * log2(e) - m two at a time; row sum in 4 packed partial sums.
           float rs8[8];
 #pragma unroll
           for (int a = 0; a < 8; ++a) rs8[a] = 0.f;
+          const float sl = p.scale_log2, nm = -m;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             uint32_t pk[16];
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-              const float p0 = ptx::ex2(fmaf(__uint_as_float(sr[j][2 * c]), p.scale_log2, -m));
-              const float p1 =
-                  ptx::ex2(fmaf(__uint_as_float(sr[j][2 * c + 1]), p.scale_log2, -m));
-              rs8[c & 7] += p0 + p1;
+              float x0, x1;
+              ptx::ffma2(x0, x1, __uint_as_float(sr[j][2 * c]), __uint_as_float(sr[j][2 * c + 1]),
+                         sl, sl, nm, nm);
+              // One pair in eight goes through the FMA-pipe polynomial, the rest
+              // through the exp unit (measured best split on B200).
+              const bool poly = (c & 7) == 7;
+              const float p0 = poly ? ptx::exp2_poly(x0) : ptx::ex2(x0);
+              const float p1 = poly ? ptx::exp2_poly(x1) : ptx::ex2(x1);
+              const int a = (c & 3) * 2;
+              ptx::fadd2(rs8[a], rs8[a + 1], rs8[a], rs8[a + 1], p0, p1);
               pk[c] = ptx::pack_bf16x2(p0, p1);
             }
             ptx::tmem_st16(tS + 64 + j * 16, pk);
           }
           const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) +
                            ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+
           lsum = lsum * alpha + rs;
           if (__any_sync(0xffffffffu, need && kt > 0)) {
 #pragma unroll

@@ -172,6 +172,11 @@ bool encode_blhd(CUtensorMap* map, const void* base, const Derived& d) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+__global__ void exp2_probe_kernel(const float* x, float* y, int n, int poly) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = poly ? sa::ptx::exp2_poly(x[i]) : sa::ptx::ex2(x[i]);
+}
+
 }  // namespace
 
 struct sa_handle {
@@ -662,6 +667,22 @@ SA_API int sa_debug_attend_simt(sa_handle* h, const void* Q, const void* Kc, con
 SA_API int sa_attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
                              int step_is_final, void* O, float* lse, sa_stream stream) {
   return attend_noalloc(h, Q, Kc, Vc, step_is_final, O, lse, stream);
+}
+
+SA_API int sa_debug_exp2(int use_polynomial, const float* x, float* y, int n, sa_stream stream) {
+  if (x == nullptr || y == nullptr || n < 0) {
+    g_error = "x and y must be non-NULL and n >= 0";
+    return SA_ERR_INVALID_ARG;
+  }
+  if (n == 0) return SA_OK;
+  exp2_probe_kernel<<<(n + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      x, y, n, use_polynomial ? 1 : 0);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    g_error = std::string("exp2 probe launch: ") + cudaGetErrorString(e);
+    return SA_ERR_CUDA;
+  }
+  return SA_OK;
 }
 
 SA_API int sa_chunk_count(const sa_handle* h, int tier) {

@@ -176,6 +176,13 @@ SA_API int sa_attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const 
 SA_API int sa_debug_attend_simt(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
                                 int step_is_final, void* O, float* lse, sa_stream stream);
 
+/* Evaluate the attention kernel's device exponentials on n fp32 values (device
+ * pointers x, y): use_polynomial = 0 -> the exp unit (ex2.approx), 1 -> the
+ * FMA-pipe polynomial 2^x used for part of the softmax (degree-3 minimax fit,
+ * relative error <= 7.5e-5 for x >= -125; x below -125 gives 2^-125). A test
+ * hook for the kernel's arithmetic; asynchronous on `stream`. */
+SA_API int sa_debug_exp2(int use_polynomial, const float* x, float* y, int n, sa_stream stream);
+
 /* Chunks appended so far to `tier`, or a negative sa_status. */
 SA_API int sa_chunk_count(const sa_handle* h, int tier);
 
