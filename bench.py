@@ -44,6 +44,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="refiner_720p")
     ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--sparsity", type=float, default=0.0,
+                    help="block-sparse mode: share of 128x128 blocks skipped (seeded random mask)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
@@ -241,35 +243,67 @@ def run_reference(args, w):
     return 0
 
 
+# ------------------------------------------------------------------ ranks
+
+
+class Ranks:
+    """Rank plumbing of a torchrun launch (also runs on CPU with gloo in tests).
+
+    Every rank takes the same collective steps in the same order: a barrier
+    around the timed region and one max-reduction per reported time.
+    """
+
+    def __init__(self, backend="nccl", device=None, timeout_s=120):
+        import torch.distributed as dist
+
+        self.dist = dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.device = device
+        if self.world > 1:
+            kw = {"device_id": device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max(self, x):
+        """Max of a float over ranks (the slowest rank's time)."""
+        import torch
+
+        t = torch.tensor([float(x)], dtype=torch.float64, device=self.device)
+        if self.world > 1:
+            self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1:
+            self.dist.destroy_process_group()
+
+
+def whole_job_tflops(flops_per_rank, ms_max, world):
+    """Aggregate throughput: the work of all ranks over the slowest rank's time."""
+    return flops_per_rank * world / (ms_max * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ GPU leg
 
 
 def run_ours(args, w):
     import torch
-    import torch.distributed as dist
 
     import block_causal_streaming_sa_b200 as sa
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks("nccl", dev)
+    world, rank = ranks.world, ranks.rank
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     stream = torch.cuda.Stream(device=dev)
     names = ("Q", "Kc", "Vc", "Kn", "Vn", "Kcl", "Vcl")
@@ -294,6 +328,21 @@ def run_ours(args, w):
             sa.sa_append_chunk(h, sa.SA_TIER_NOISY, s["Kn"].data_ptr(), s["Vn"].data_ptr(), sp)
             sa.sa_append_chunk(h, sa.SA_TIER_CLEAN, s["Kcl"].data_ptr(), s["Vcl"].data_ptr(), sp)
 
+    block_mask = None
+    if args.sparsity > 0:
+        # Steady-state chunk: S + W attended chunks; a seeded mask with the given share
+        # of 128x128 blocks skipped. FLOPs count only the flagged blocks.
+        nq = -(-w.chunk_len // 128)
+        nk = (w.sink + w.window) * nq
+        gen = torch.Generator().manual_seed(1234)
+        block_mask = (torch.rand((w.batch, w.heads, nq, nk), generator=gen) >= args.sparsity)
+        rows = torch.full((nq,), 128.0)
+        rows[-1] = w.chunk_len - 128 * (nq - 1)
+        keys = rows.repeat(w.sink + w.window)
+        flops = float(4.0 * w.head_dim * (block_mask.double() * rows[:, None].double()
+                                          * keys[None, :].double()).sum())
+        block_mask = block_mask.to(torch.uint8).to(dev)
+
     def chunk_step(s, ev=None):
         """One chunk: every denoising step's attention in every layer, then the appends."""
         a = 0
@@ -301,11 +350,19 @@ def run_ours(args, w):
             final = k == steps_per_chunk - 1
             for layer in layers:
                 h = layer.handle
-                sa.sa_stage_keys(h, s["Kc"].data_ptr(), sp)
-                if ev is not None:
-                    ev[0][a].record(stream)
-                sa.sa_attend_staged(h, s["Q"].data_ptr(), s["Vc"].data_ptr(), final,
-                                    out.data_ptr(), 0, sp)
+                if block_mask is not None:
+                    # sparse: the staging kernel is inside the timed attention call
+                    if ev is not None:
+                        ev[0][a].record(stream)
+                    sa.sa_attend_sparse(h, s["Q"].data_ptr(), s["Kc"].data_ptr(),
+                                        s["Vc"].data_ptr(), final, block_mask.data_ptr(),
+                                        out.data_ptr(), 0, sp)
+                else:
+                    sa.sa_stage_keys(h, s["Kc"].data_ptr(), sp)
+                    if ev is not None:
+                        ev[0][a].record(stream)
+                    sa.sa_attend_staged(h, s["Q"].data_ptr(), s["Vc"].data_ptr(), final,
+                                        out.data_ptr(), 0, sp)
                 if ev is not None:
                     ev[1][a].record(stream)
                 a += 1
@@ -370,16 +427,14 @@ def run_ours(args, w):
 
     ms_max = max_over_ranks(ms_local)
     e2e_ms_max = max_over_ranks(e2e_ms_local)
-    total_flops = flops * attends_per_chunk * args.steps * world
-    value = total_flops / (ms_max * 1e-3) / 1e12
-    e2e_value = flops * attends_per_chunk * e2e_steps * world / (e2e_ms_max * 1e-3) / 1e12
+    value = whole_job_tflops(flops * attends_per_chunk * args.steps, ms_max, world)
+    e2e_value = whole_job_tflops(flops * attends_per_chunk * e2e_steps, e2e_ms_max, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.cpu_seconds)
 
-    if world > 1:
-        dist.destroy_process_group()
+    ranks.close()
     if rank != 0:
         return 0
 
@@ -413,9 +468,12 @@ def run_ours(args, w):
             "l2": f"inputs larger than L2: {cache_bytes_read / 2**20:.0f} MiB of cached K/V "
                   f"read per attention vs {L2_BYTES / 2**20:.0f} MiB L2",
             "parallelism": f"replicas{world}" if world > 1 else "single",
+            "block_sparsity": args.sparsity,
         },
         "roofline": {
-            "bound": "tensor", "kernel": "attend_tc_kernel<128>",
+            "bound": "tensor",
+            "kernel": "attend_tc_kernel<128>" + (" (sparse, timed with its staging kernel)"
+                                                 if block_mask is not None else ""),
             "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "peak_kind": f"bf16 sustained ({peak_src})", "frac_of_burst_peak": achieved / burst,
             "traffic": kernel_traffic("attend_tc.cuh", w.name),

@@ -66,6 +66,9 @@ _SIGNATURES = {
     "sa_debug_attend_simt": (_I, [_P, _P, _P, _P, _I, _P, _P, _P]),
     "sa_attend_noalloc": (_I, [_P, _P, _P, _P, _I, _P, _P, _P]),
     "sa_debug_exp2": (_I, [_I, _P, _P, _I, _P]),
+    "sa_attend_sparse": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P]),
+    "sa_block_grid": (_I, [_CFGP, ctypes.c_int32, _I32P, _I32P]),
+    "sa_debug_attend_stalled": (_I, [_P, _P, _P, _P, _I, _P, _P]),
     "sa_chunk_count": (_I, [_P, _I]),
     "sa_debug_layout": (_I, [_P, _I, _I32P, _I]),
     "sa_plan": (_I, [_CFGP, ctypes.c_int32, _I32P, _I32P, _I32P, _I]),
@@ -167,6 +170,22 @@ def sa_attend_noalloc(handle, Q, Kc, Vc, step_is_final, O, lse=0, stream=0):
     the library (for callers that cannot allocate device memory)."""
     _check(lib().sa_attend_noalloc(handle, _P(Q), _P(Kc), _P(Vc), int(bool(step_is_final)),
                                    _P(O), _P(lse or None), _P(stream)), handle)
+
+
+def sa_attend_sparse(handle, Q, Kc, Vc, step_is_final, block_mask, O, lse=0, stream=0):
+    _check(lib().sa_attend_sparse(handle, _P(Q), _P(Kc), _P(Vc), int(bool(step_is_final)),
+                                  _P(block_mask), _P(O), _P(lse or None), _P(stream)), handle)
+
+
+def sa_block_grid(cfg, chunk):
+    nq, nk = ctypes.c_int32(), ctypes.c_int32()
+    _check(lib().sa_block_grid(ctypes.byref(cfg), chunk, ctypes.byref(nq), ctypes.byref(nk)))
+    return nq.value, nk.value
+
+
+def sa_debug_attend_stalled(handle, Q, Kc, Vc, step_is_final, O, stream=0):
+    _check(lib().sa_debug_attend_stalled(handle, _P(Q), _P(Kc), _P(Vc), int(bool(step_is_final)),
+                                         _P(O), _P(stream)), handle)
 
 
 def sa_debug_exp2(use_polynomial, x, y, n, stream=0):

@@ -4,19 +4,21 @@
 // 「实时」改变了什么 and 选择三：有上限的记忆): for every query row of the chunk
 // being generated, softmax attention over the keys of the cached sink and window
 // chunks of one TwinCache tier plus the chunk's own keys, with the temporal RoPE
-// position of chunk j relocated to rank(j) * F.
+// position of chunk j relocated to rank(j) * F. With kSparse, only the 128 x 128
+// blocks a caller flags are attended (section 选择四：速度从哪里来: block-sparse
+// attention with most blocks skipped).
 //
 // Design (B200):
 //  * persistent CTAs, one per SM; a work tile is two 128-row query tiles of one
 //    (batch, head), so every K/V tile brought in by TMA feeds two MMAs;
-//  * warp 0 (one lane): TMA producer over a ring of NSTAGE 128x D bf16 tiles,
+//  * warp 0 (one lane): TMA producer over a ring of NSTAGE 128x D tiles,
 //    K_0 V_0 K_1 V_1 ..., 128-byte swizzle, straight from the cache slots and
 //    from the caller's V (no gather copy);
-//  * warp 1 (one lane): tcgen05.mma issuer. S_i = Q_i K^T (SS form, both
-//    operands K-major in shared memory) into TMEM, then O_i += P_i V (TS form:
-//    P_i read from TMEM, written over the upper half of S_i, V MN-major in shared memory);
-//    the two query tiles ping-pong so one tile's softmax overlaps the other's
-//    MMAs;
+//  * warp 1 (one lane): tcgen05.mma issuer. S_i = Q_i K^T (SS form, fp16, both
+//    operands K-major in shared memory) into TMEM, then O_i += P_i V (TS form,
+//    bf16: P_i read from TMEM, written over the upper half of S_i, V MN-major
+//    in shared memory); the two query tiles ping-pong so one tile's softmax
+//    overlaps the other's MMAs;
 //  * warps 4-7 / 8-11: one warpgroup per query tile, thread = query row =
 //    TMEM lane. Each writes its rotated query tile into shared memory, runs the
 //    online softmax on S rows read from TMEM in one round trip (no cross-thread
@@ -24,15 +26,20 @@
 //    maxima, scale-and-subtract and the row sum in packed fp32x2 instructions,
 //    1 exponential in 8 on the FMA pipe by a fitted polynomial), writes P
 //    back as bf16, rescales O in TMEM only when the running max grows by more
-//    than 2^8, and runs the epilogue;
+//    than 2^8, and calls the epilogue;
 //  * registers: launched at 168 per thread (384 threads), warpgroup 0 (warps
 //    0-3: producer, MMA issuer, two idle) gives registers back with setmaxnreg
 //    (104) and the softmax warpgroups take them (200), so a whole 128-score row
-//    stays in registers without spills;
+//    stays in registers without spills; the epilogue is a separate function so
+//    its registers do not add to the score loop's;
 //  * RoPE: keys are stored rotated by their in-chunk position; the relocated
 //    temporal base rank(j) * F of the attended chunk is applied by re-turning
 //    the temporal band of the query tile when the key stream moves to the next
-//    chunk, before the first QK^T MMA of that chunk.
+//    chunk, before the first QK^T MMA of that chunk;
+//  * work units: rounds of gridDim.x work tiles; when the last round holds at
+//    most half a grid of tiles, each of them is split by attended chunks into
+//    two halves run by two CTAs, which write normalised fp32 partial rows and
+//    their log-sum-exp; per row, the second half to finish merges both.
 // All mbarrier waits are bounded (see ptx.cuh); on a timeout every role drains
 // its outstanding async work, TMEM is freed and the device status word is set.
 #pragma once
@@ -59,8 +66,8 @@ struct TcShape {
   // Register split (setmaxnreg): launched at kLaunchRegs per thread (the
   // __launch_bounds__(384, 1) budget); warpgroup 0 (producer, MMA) drops to
   // kRegsCtl, the two softmax warpgroups rise to kRegsSoftmax.
-  // 128 * 56 + 256 * 224 = 64512 = 384 * 168 (the launch pool), and per SM
-  // sub-partition 56 + 224 + 224 = 504 <= 512 registers per thread slot.
+  // 128 * 104 + 256 * 200 = 64512 = 384 * 168 (the launch pool), and per SM
+  // sub-partition 104 + 200 + 200 = 504 <= 512 registers per thread slot.
   static constexpr int kLaunchRegs = 168;
   static constexpr int kRegsCtl = 104;
   static constexpr int kRegsSoftmax = 200;
@@ -70,14 +77,13 @@ struct TcShape {
   static constexpr int kOffQRaw = kOffKV + NSTAGE * kTile;  // raw temporal chunks of both Q tiles
   static constexpr int kQRawRow = ((D - 4 * (D / 6) + 7) / 8) * 16;
   static constexpr int kOffBar = kOffQRaw + 2 * BM * kQRawRow;
-  static constexpr int kOffGroups = kOffBar + 256;          // attended-chunk table
-  static constexpr int kSmemBytes = kOffGroups + 256 + 1024;  // + table + alignment slack
+  static constexpr int kOffGroups = kOffBar + 256;  // attended-chunk table, tile starts, schedule
+  static constexpr int kSmemBytes = kOffGroups + 256 + 128 + 1024;  // + alignment slack
   static constexpr int kTmemCols = 512;
   static constexpr int kDt = D - 4 * (D / 6);             // temporal band width
   static constexpr int kTChunks = (kDt + 7) / 8;           // 16-byte chunks holding it
   static constexpr uint32_t kIdescQK = ptx::idesc_f32acc(BM, BN, 0, 0);  // fp16 Q~, K~
   static constexpr uint32_t kIdescPV = ptx::idesc_f32acc(BM, D, 1, 1);   // bf16 P, V
-
   __host__ __device__ static constexpr int col_s(int i) { return i * 128; }
   __host__ __device__ static constexpr int col_o(int i) { return 256 + i * D; }
   __host__ __device__ static constexpr int col_p(int i) { return i * 128 + 64; }  // bf16 P
@@ -114,7 +120,106 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   return v;
 }
 
+// Epilogue of one query row of a work unit; a function of its own so that its
+// registers do not count against the score loop's (it runs once per unit).
+// O / l -> bf16 row of [B, L, H, D] and the natural-log LSE; a row that saw no
+// key (every block unflagged) gets O = 0 and lse = -inf. For a chunk-range half
+// of a split tile (half >= 0): write the normalised fp32 partial row and its
+// lse; the second of the two halves to finish (per-row counter) merges the two
+// in half order, so the result does not depend on timing.
 template <int D>
+__device__ __noinline__ void epilogue(const AttendParams& p, uint32_t tO, bool any_tile, float m,
+                                      float lsum, int half, int slot, int i, int r,
+                                      unsigned long long row_off, long long lse_idx, bool valid) {
+  using T = TcShape<D>;
+  const bool seen = lsum > 0.f;
+  const float inv = seen ? 1.f / lsum : 0.f;
+  const float lse_own = seen ? (m + __log2f(lsum)) * 0.69314718055994531f : -INFINITY;
+  uint4* dst = reinterpret_cast<uint4*>(p.o + row_off);
+  if (half < 0) {
+#pragma unroll 1
+    for (int j = 0; j < D / 32; ++j) {
+      uint32_t o[32];
+      if (any_tile) {
+        ptx::tmem_ld32(tO + j * 32, o);
+        ptx::tmem_wait_ld();
+      }
+      if (valid) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint4 q4 = make_uint4(0u, 0u, 0u, 0u);
+          if (seen) {
+            q4.x = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv,
+                                    __uint_as_float(o[8 * v + 1]) * inv);
+            q4.y = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv,
+                                    __uint_as_float(o[8 * v + 3]) * inv);
+            q4.z = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv,
+                                    __uint_as_float(o[8 * v + 5]) * inv);
+            q4.w = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv,
+                                    __uint_as_float(o[8 * v + 7]) * inv);
+          }
+          st_v4(dst + j * 4 + v, q4);
+        }
+      }
+    }
+    if (valid && p.lse != nullptr) p.lse[lse_idx] = lse_own;
+    return;
+  }
+  const size_t prow = ((static_cast<size_t>(slot) * 2 + i) * 2 + half) * T::BM + r;
+  const size_t qrow = ((static_cast<size_t>(slot) * 2 + i) * 2 + (1 - half)) * T::BM + r;
+  float* po = p.split_o + prow * D;
+#pragma unroll 1
+  for (int j = 0; j < D / 32; ++j) {
+    uint32_t o[32];
+    if (any_tile) {
+      ptx::tmem_ld32(tO + j * 32, o);
+      ptx::tmem_wait_ld();
+    }
+#pragma unroll
+    for (int c = 0; c < 32; c += 4)
+      reinterpret_cast<float4*>(po + j * 32)[c / 4] =
+          seen ? make_float4(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv,
+                             __uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv)
+               : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  p.split_lse[prow] = lse_own;
+  __threadfence();
+  int* sem = p.split_sem + (static_cast<size_t>(slot) * 2 + i) * T::BM + r;
+  if (atomicAdd(sem, 1) != 1) return;  // the other half merges
+  __threadfence();
+  const float lse_other = __ldcg(p.split_lse + qrow);
+  const float l0 = half == 0 ? lse_own : lse_other;
+  const float l1 = half == 0 ? lse_other : lse_own;
+  const float* o0 = half == 0 ? po : p.split_o + qrow * D;
+  const float* o1 = half == 0 ? p.split_o + qrow * D : po;
+  const float mx2 = fmaxf(l0, l1);
+  float w0 = 0.f, w1 = 0.f, lse_tot = -INFINITY;
+  if (mx2 != -INFINITY) {
+    const float e0 = __expf(l0 - mx2), e1 = __expf(l1 - mx2);
+    lse_tot = mx2 + __logf(e0 + e1);
+    w0 = e0 / (e0 + e1);
+    w1 = e1 / (e0 + e1);
+  }
+  if (valid) {
+#pragma unroll 1
+    for (int c = 0; c < D; c += 8) {
+      const float4 a0 = __ldcg(reinterpret_cast<const float4*>(o0 + c));
+      const float4 a1 = __ldcg(reinterpret_cast<const float4*>(o0 + c + 4));
+      const float4 b0 = __ldcg(reinterpret_cast<const float4*>(o1 + c));
+      const float4 b1 = __ldcg(reinterpret_cast<const float4*>(o1 + c + 4));
+      uint4 q4;
+      q4.x = ptx::pack_bf16x2(fmaf(w1, b0.x, w0 * a0.x), fmaf(w1, b0.y, w0 * a0.y));
+      q4.y = ptx::pack_bf16x2(fmaf(w1, b0.z, w0 * a0.z), fmaf(w1, b0.w, w0 * a0.w));
+      q4.z = ptx::pack_bf16x2(fmaf(w1, b1.x, w0 * a1.x), fmaf(w1, b1.y, w0 * a1.y));
+      q4.w = ptx::pack_bf16x2(fmaf(w1, b1.z, w0 * a1.z), fmaf(w1, b1.w, w0 * a1.w));
+      st_v4(dst + c / 8, q4);
+    }
+    if (p.lse != nullptr) p.lse[lse_idx] = lse_tot;
+  }
+  *sem = 0;  // ready for the next launch
+}
+
+template <int D, bool kSparse>
 __global__ void __launch_bounds__(384, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tm_cache,
                      const __grid_constant__ CUtensorMap tm_kcur,
@@ -132,13 +237,33 @@ __global__ void __launch_bounds__(384, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // The attended-chunk table, indexed by a runtime chunk counter, lives in shared
-  // memory (dynamic indexing of a kernel parameter would copy it to local memory).
+  const int n_qt = (p.L + T::BM - 1) / T::BM;
+  const int n_pairs = (n_qt + 1) / 2;
+  const int n_work = p.B * p.H * n_pairs;
+
+  // Shared tables (dynamic indexing of a kernel parameter would copy it to local
+  // memory): the attended chunks, the first key tile of each, and the schedule
+  // sched = {rounds, tail, split, middle chunk} of the work units.
   AttendGroup* groups = reinterpret_cast<AttendGroup*>(smem + T::kOffGroups);
+  int* gstart = reinterpret_cast<int*>(smem + T::kOffGroups + 256);
+  volatile int* sched = reinterpret_cast<volatile int*>(smem + T::kOffGroups + 256 + 72);
   static_assert(sizeof(AttendGroup) * kMaxGroups <= 256, "group table");
   if (threadIdx.x == 0) {
+    int acc = 0;
 #pragma unroll
-    for (int g = 0; g < kMaxGroups; ++g) groups[g] = p.groups[g];
+    for (int g = 0; g < kMaxGroups; ++g) {
+      groups[g] = p.groups[g];
+      gstart[g] = acc;
+      if (g < p.n_groups) acc += (p.groups[g].len + T::BN - 1) / T::BN;
+    }
+    gstart[kMaxGroups] = acc;
+    const int rounds = (n_work + gridDim.x - 1) / gridDim.x;
+    const int tail = n_work - (rounds - 1) * gridDim.x;
+    sched[0] = rounds;
+    sched[1] = tail;
+    sched[2] = p.split_ok && p.n_groups >= 2 && 2 * tail <= static_cast<int>(gridDim.x) &&
+               tail <= kMaxSplitSlots;
+    sched[3] = p.n_groups / 2;
   }
 
   if (threadIdx.x == 0) {
@@ -164,31 +289,68 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+  const int n_kt_total = gstart[p.n_groups];
 
-  const int n_qt = (p.L + T::BM - 1) / T::BM;
-  const int n_pairs = (n_qt + 1) / 2;
-  const int n_work = p.B * p.H * n_pairs;
-  int n_kt_total = 0;
-  for (int g = 0; g < p.n_groups; ++g) n_kt_total += (groups[g].len + T::BN - 1) / T::BN;
+  // Work unit r of this CTA: work tile w over attended chunks [g_lo, g_hi).
+  // half = -1 for a whole tile, 0 / 1 for the two halves of a split tail tile.
+  auto unit = [&](int r, int& w, int& half) -> bool {
+    const int rounds = sched[0];
+    half = -1;
+    if (!sched[2] || r < rounds - 1) {
+      w = blockIdx.x + r * gridDim.x;
+      return w < n_work;
+    }
+    if (r > rounds - 1 || static_cast<int>(blockIdx.x) >= 2 * sched[1]) return false;
+    w = (rounds - 1) * gridDim.x + (blockIdx.x >> 1);
+    half = blockIdx.x & 1;
+    return true;
+  };
+  auto g_lo = [&](int half) { return half == 1 ? sched[3] : 0; };
+  auto g_hi = [&](int half) { return half == 0 ? sched[3] : p.n_groups; };
+
+  // Block sparsity: key tile kt of a work tile is visited when either of its two
+  // query tiles has the block flagged. Flag rows at mask offsets mo (query tile
+  // 2 * pair) and mo1 (its partner, -1 when the pair has a single tile).
+  auto mask_rows = [&](int w, int& mo, int& mo1) {
+    mo = mo1 = -1;
+    if (!kSparse) return;
+    const int bh = w / n_pairs, pair = w - bh * n_pairs;
+    mo = (bh * n_qt + 2 * pair) * n_kt_total;
+    mo1 = 2 * pair + 1 < n_qt ? mo + n_kt_total : -1;
+  };
+  auto flag = [&](int off, int kt) -> bool {
+    return off >= 0 && __ldg(p.block_mask + off + kt) != 0;
+  };
+  auto next_visited = [&](int mo, int mo1, int from, int hi) {
+    if (!kSparse) return from;
+    int kt = from;
+    while (kt < hi && !(flag(mo, kt) || flag(mo1, kt))) ++kt;
+    return kt;
+  };
 
   if (warp < 4) {
   ptx::setmaxnreg_dec<T::kRegsCtl>();
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    if (lane == 0 && !p.debug_stall_producer) {
       ptx::tma_prefetch_desc(&tm_cache);
       ptx::tma_prefetch_desc(&tm_kcur);
       ptx::tma_prefetch_desc(&tm_vcur);
       int stage = 0;
       uint32_t phase = 0, filled_mask = 0, filled_parity = 0;
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x) {
+      for (int rr = 0; ok; ++rr) {
+        int w, half;
+        if (!unit(rr, w, half)) break;
         const int bh = w / n_pairs;
         const int b = bh / p.H, h = bh - b * p.H;
-        for (int g = 0; ok && g < p.n_groups; ++g) {
+        int mo, mo1;
+        mask_rows(w, mo, mo1);
+        for (int g = g_lo(half); ok && g < g_hi(half); ++g) {
           const AttendGroup grp = groups[g];
           const int nkt = (grp.len + T::BN - 1) / T::BN;
           for (int t = 0; ok && t < nkt; ++t) {
+            if (kSparse && !(flag(mo, gstart[g] + t) || flag(mo1, gstart[g] + t))) continue;
             for (int kv = 0; kv < 2; ++kv) {
               if (!ptx::mbar_wait(bar(T::EMPTY(stage)), phase ^ 1u, abort_flag, p.status)) {
                 ok = false;
@@ -259,13 +421,23 @@ __global__ void __launch_bounds__(384, 1)
                        (accumulate || kk > 0) ? 1u : 0u);
         }
       };
-      int wi = 0;
-      for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++wi) {
+      for (int rr = 0; ok; ++rr) {
+        int w, half;
+        if (!unit(rr, w, half)) break;
+        const int lo = gstart[g_lo(half)], hi = gstart[g_hi(half)];
+        int mo, mo1;
+        mask_rows(w, mo, mo1);
+        int u = next_visited(mo, mo1, lo, hi);
+        if (kSparse && u >= hi) {  // no block flagged: nothing to multiply
+          for (int i = 0; i < 2 && ok; ++i)
+            ok = ptx::mbar_wait(bar(T::QREADY(i)), rr & 1, abort_flag, p.status);
+          continue;
+        }
         int sk = 0, sv = 0;
         if (!take_stage(sk)) break;
         ptx::tc_fence_after();
         for (int i = 0; i < 2; ++i) {
-          if (!ptx::mbar_wait(bar(T::QREADY(i)), wi & 1, abort_flag, p.status)) {
+          if (!ptx::mbar_wait(bar(T::QREADY(i)), rr & 1, abort_flag, p.status)) {
             ok = false;
             break;
           }
@@ -275,8 +447,9 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (!ok) break;
         ptx::umma_commit(bar(T::EMPTY(sk)));
-        for (int kt = 0; ok && kt < n_kt_total; ++kt) {
-          const bool has_next = kt + 1 < n_kt_total;
+        for (bool first = true; ok && u < hi; first = false) {
+          const int nu = next_visited(mo, mo1, u + 1, hi);
+          const bool has_next = nu < hi;
           if (!take_stage(sv) || (has_next && !take_stage(sk))) {
             ok = false;
             break;
@@ -289,7 +462,7 @@ __global__ void __launch_bounds__(384, 1)
             }
             pf_phase[i] ^= 1u;
             ptx::tc_fence_after();
-            issue_pv(i, sv, kt > 0);
+            issue_pv(i, sv, !first);
             if (i == 1) ptx::umma_commit(bar(T::EMPTY(sv)));
             if (!has_next) ptx::umma_commit(bar(T::OFINAL(i)));
             if (has_next) {
@@ -298,6 +471,7 @@ __global__ void __launch_bounds__(384, 1)
             }
           }
           if (ok && has_next) ptx::umma_commit(bar(T::EMPTY(sk)));
+          u = nu;
         }
       }
       // Every MMA issued so far must finish before TMEM is released.
@@ -318,8 +492,10 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t q_smem = sbase + T::kOffQ + i * T::kTile;
     uint32_t s_phase = 0;
     bool ok = true;
-    int wi = 0;
-    for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++wi) {
+    int o_units = 0;  // units whose O this warpgroup waited for (OFINAL phases)
+    for (int rr = 0; ok; ++rr) {
+      int w, half;
+      if (!unit(rr, w, half)) break;
       const int bh = w / n_pairs, pair = w - bh * n_pairs;
       const int b = bh / p.H, h = bh - b * p.H;
       const int q_row = (2 * pair + i) * T::BM + r;
@@ -329,13 +505,27 @@ __global__ void __launch_bounds__(384, 1)
       const int y = (qr / p.rope.tok_w) % p.rope.tok_h;
       const int x = qr % p.rope.tok_w;
       const size_t row_off = ((static_cast<size_t>(b) * p.L + qr) * p.H + h) * D;
+      const int glo = g_lo(half), ghi = g_hi(half);
+      int mo = -1, mo1 = -1, own = -1;
+      if (kSparse) {
+        mask_rows(w, mo, mo1);
+        own = i == 0 ? mo : mo1;
+      }
+      // First chunk with a visited key tile (the query tile is rotated for it).
+      int g0 = glo;
+      bool any_tile = true;
+      if (kSparse) {
+        const int u0 = next_visited(mo, mo1, gstart[glo], gstart[ghi]);
+        any_tile = u0 < gstart[ghi];
+        while (g0 + 1 < ghi && u0 >= gstart[g0 + 1]) ++g0;
+      }
 
-      // Rotated query tile for the first attended chunk; the raw temporal chunks
-      // are kept in shared memory for the re-turns at chunk switches.
+      // Rotated query tile for that chunk; the raw temporal chunks are kept in
+      // shared memory for the re-turns at chunk switches.
       const uint32_t q_raw = sbase + T::kOffQRaw + (i * T::BM + r) * T::kQRawRow;
       {
         const uint4* src = reinterpret_cast<const uint4*>(p.q + row_off);
-        const int td0 = groups[0].t_delta;
+        const int td0 = groups[g0].t_delta;
 #pragma unroll 2
         for (int c = 0; c < D / 8; ++c) {
           uint4 v = valid ? ld_nc_v4(src + c) : make_uint4(0u, 0u, 0u, 0u);
@@ -347,93 +537,116 @@ __global__ void __launch_bounds__(384, 1)
       }
 
       float m = -INFINITY, lsum = 0.f;
-      int kt = 0;
-      for (int g = 0; ok && g < p.n_groups; ++g) {
+      int kt = 0;  // key tiles processed in this unit
+      for (int g = glo; ok && any_tile && g < ghi; ++g) {
         const int len = groups[g].len;
         const int nkt = (len + T::BN - 1) / T::BN;
-        for (int t = 0; t < nkt; ++t, ++kt) {
+        for (int t = 0; t < nkt; ++t) {
+          if (kSparse && next_visited(mo, mo1, gstart[g] + t, gstart[g] + t + 1) != gstart[g] + t)
+            continue;
           if (!ptx::mbar_wait(bar(T::SFULL(i)), s_phase, abort_flag, p.status)) {
             ok = false;
             break;
           }
           s_phase ^= 1u;
           ptx::tc_fence_after();
-          // The whole score row (128 fp32) in one round trip; keys past the chunk end masked.
-          const int nvalid = min(T::BN, len - t * T::BN);
-          uint32_t sr[4][32];
+          if (!kSparse || flag(own, gstart[g] + t)) {
+            // The whole score row (128 fp32) in one round trip; keys past the chunk end masked.
+            const int nvalid = min(T::BN, len - t * T::BN);
+            uint32_t sr[4][32];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) ptx::tmem_ld32(tS + j * 32, sr[j]);
-          ptx::tmem_wait_ld();
-          if (nvalid < T::BN) {
+            for (int j = 0; j < 4; ++j) ptx::tmem_ld32(tS + j * 32, sr[j]);
+            ptx::tmem_wait_ld();
+            if (nvalid < T::BN) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                  if (j * 32 + c >= nvalid) sr[j][c] = __float_as_uint(-INFINITY);
+            }
+            // Row max as a tree over 8 independent running maxima (3-input max).
+            float mx8[8];
+#pragma unroll
+            for (int a = 0; a < 8; ++a) mx8[a] = __uint_as_float(sr[0][a]);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
 #pragma unroll
-              for (int c = 0; c < 32; ++c)
-                if (j * 32 + c >= nvalid) sr[j][c] = __float_as_uint(-INFINITY);
-          }
-          // Row max as a tree over 8 independent running maxima (3-input max).
-          float mx8[8];
-#pragma unroll
-          for (int a = 0; a < 8; ++a) mx8[a] = __uint_as_float(sr[0][a]);
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int c = 0; c < 32; c += 2)
-              if (j > 0 || c >= 8)
-                mx8[(c >> 1) & 7] = ptx::fmax3(mx8[(c >> 1) & 7], __uint_as_float(sr[j][c]),
-                                               __uint_as_float(sr[j][c + 1]));
-          const float mx = fmaxf(ptx::fmax3(mx8[0], mx8[1], mx8[2]),
-                                 fmaxf(ptx::fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-          const float m_new = fmaxf(m, mx * p.scale_log2);
-          const bool need = m_new > m + 8.0f;
-          float alpha = 1.f;
-          if (need) {
-            alpha = ptx::ex2(m - m_new);
-            m = m_new;
-          }
-          // P = 2^(s * scale * log2 e - m) as bf16 pairs in columns 64..127 of the S
-          // region (P of key k in column 64 + k / 2); the sum over 8 partial sums.
-          // x = s * scale * log2(e) - m two at a time; row sum in 4 packed partial sums.
-          float rs8[8];
-#pragma unroll
-          for (int a = 0; a < 8; ++a) rs8[a] = 0.f;
-          const float sl = p.scale_log2, nm = -m;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              float x0, x1;
-              ptx::ffma2(x0, x1, __uint_as_float(sr[j][2 * c]), __uint_as_float(sr[j][2 * c + 1]),
-                         sl, sl, nm, nm);
-              // One pair in eight goes through the FMA-pipe polynomial, the rest
-              // through the exp unit (measured best split on B200).
-              const bool poly = (c & 7) == 7;
-              const float p0 = poly ? ptx::exp2_poly(x0) : ptx::ex2(x0);
-              const float p1 = poly ? ptx::exp2_poly(x1) : ptx::ex2(x1);
-              const int a = (c & 3) * 2;
-              ptx::fadd2(rs8[a], rs8[a + 1], rs8[a], rs8[a + 1], p0, p1);
-              pk[c] = ptx::pack_bf16x2(p0, p1);
+              for (int c = 0; c < 32; c += 2)
+                if (j > 0 || c >= 8)
+                  mx8[(c >> 1) & 7] = ptx::fmax3(mx8[(c >> 1) & 7], __uint_as_float(sr[j][c]),
+                                                 __uint_as_float(sr[j][c + 1]));
+            const float mx =
+                fmaxf(ptx::fmax3(mx8[0], mx8[1], mx8[2]),
+                      fmaxf(ptx::fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            const float m_new = fmaxf(m, mx * p.scale_log2);
+            const bool need = m_new > m + 8.0f;
+            float alpha = 1.f;
+            if (need) {
+              alpha = ptx::ex2(m - m_new);
+              m = m_new;
             }
-            ptx::tmem_st16(tS + 64 + j * 16, pk);
-          }
-          const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) +
-                           ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
-
-          lsum = lsum * alpha + rs;
-          if (__any_sync(0xffffffffu, need && kt > 0)) {
+            // P = 2^(s * scale * log2 e - m) as bf16 pairs in columns 64..127 of the S
+            // region (P of key k in column 64 + k / 2). x = s * scale * log2(e) - m two
+            // at a time; the row sum in 4 packed partial sums.
+            float rs8[8];
 #pragma unroll
-            for (int j = 0; j < D / 32; ++j) {
-              uint32_t o[32];
-              ptx::tmem_ld32(tO + j * 32, o);
-              ptx::tmem_wait_ld();
+            for (int a = 0; a < 8; ++a) rs8[a] = 0.f;
+            const float sl = p.scale_log2, nm = -m;
 #pragma unroll
-              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-              ptx::tmem_st32(tO + j * 32, o);
+            for (int j = 0; j < 4; ++j) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int c = 0; c < 16; ++c) {
+                float x0, x1;
+                ptx::ffma2(x0, x1, __uint_as_float(sr[j][2 * c]),
+                           __uint_as_float(sr[j][2 * c + 1]), sl, sl, nm, nm);
+                // One pair in eight goes through the FMA-pipe polynomial, the rest
+                // through the exp unit (measured best split on B200).
+                const bool poly = (c & 7) == 7;
+                const float p0 = poly ? ptx::exp2_poly(x0) : ptx::ex2(x0);
+                const float p1 = poly ? ptx::exp2_poly(x1) : ptx::ex2(x1);
+                const int a = (c & 3) * 2;
+                ptx::fadd2(rs8[a], rs8[a + 1], rs8[a], rs8[a + 1], p0, p1);
+                pk[c] = ptx::pack_bf16x2(p0, p1);
+              }
+              ptx::tmem_st16(tS + 64 + j * 16, pk);
             }
+            const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) +
+                             ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+            lsum = lsum * alpha + rs;
+            // The first tile's P.V overwrote O; a later growth of the max rescales it.
+            if (__any_sync(0xffffffffu, need && kt > 0)) {
+#pragma unroll
+              for (int j = 0; j < D / 32; ++j) {
+                uint32_t o[32];
+                ptx::tmem_ld32(tO + j * 32, o);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                  o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                ptx::tmem_st32(tO + j * 32, o);
+              }
+            }
+          } else {
+            // Block flagged for the partner query tile only: P = 0 here.
+            uint32_t zero[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) zero[c] = 0u;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) ptx::tmem_st16(tS + 64 + j * 16, zero);
           }
-          if (t == nkt - 1 && g + 1 < p.n_groups) {
-            const int td = groups[g + 1].t_delta;
+          // Chunk switch: the next key tile lies in a later chunk; turn the query
+          // tile's temporal band to that chunk's relocated offset first.
+          int gn = g;
+          if (kSparse) {
+            const int nu = next_visited(mo, mo1, gstart[g] + t + 1, gstart[ghi]);
+            if (nu < gstart[ghi] && nu >= gstart[g + 1])
+              while (gn + 1 < ghi && nu >= gstart[gn + 1]) ++gn;
+          } else if (t == nkt - 1 && g + 1 < ghi) {
+            gn = g + 1;
+          }
+          if (gn != g) {
+            const int td = groups[gn].t_delta;
 #pragma unroll 2
             for (int c = 0; c < T::kTChunks; ++c)
               st_shared_v4(q_smem + sw128_offset(r, c),
@@ -443,39 +656,19 @@ __global__ void __launch_bounds__(384, 1)
           ptx::tmem_wait_st();
           ptx::tc_fence_before();
           ptx::mbar_arrive(bar(T::PFULL(i)));
+          ++kt;
         }
       }
       if (!ok) break;
 
-      // Epilogue: O / l -> bf16 rows of [B, L, H, D]; optional natural-log LSE.
-      if (!ptx::mbar_wait(bar(T::OFINAL(i)), wi & 1, abort_flag, p.status)) break;
-      ptx::tc_fence_after();
-      const float inv = 1.f / lsum;
-      uint4* dst = reinterpret_cast<uint4*>(p.o + row_off);
-#pragma unroll 1
-      for (int j = 0; j < D / 32; ++j) {
-        uint32_t o[32];
-        ptx::tmem_ld32(tO + j * 32, o);
-        ptx::tmem_wait_ld();
-        if (valid) {
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 u;
-            u.x = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv,
-                                   __uint_as_float(o[8 * v + 1]) * inv);
-            u.y = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv,
-                                   __uint_as_float(o[8 * v + 3]) * inv);
-            u.z = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv,
-                                   __uint_as_float(o[8 * v + 5]) * inv);
-            u.w = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv,
-                                   __uint_as_float(o[8 * v + 7]) * inv);
-            st_v4(dst + j * 4 + v, u);
-          }
-        }
+      if (any_tile) {
+        if (!ptx::mbar_wait(bar(T::OFINAL(i)), o_units & 1, abort_flag, p.status)) break;
+        ++o_units;
+        ptx::tc_fence_after();
       }
-      if (valid && p.lse != nullptr)
-        p.lse[(static_cast<size_t>(b) * p.H + h) * p.L + q_row] =
-            (m + __log2f(lsum)) * 0.69314718055994531f;
+      epilogue<D>(p, tO, any_tile, m, lsum, half,
+                  w - (sched[0] - 1) * static_cast<int>(gridDim.x), i, r, row_off,
+                  (static_cast<long long>(b) * p.H + h) * p.L + q_row, valid);
       ptx::tc_fence_before();
     }
   }

@@ -35,7 +35,8 @@ struct Derived {
   float scale, theta;
   size_t chunk_elems;  // B * H * L * D
   // byte offsets inside the device buffer
-  size_t off_status, off_rope_t, off_rope_h, off_rope_w, off_tier[2], off_kcur, total;
+  size_t off_status, off_rope_t, off_rope_h, off_rope_w, off_tier[2], off_kcur;
+  size_t off_split_o, off_split_lse, off_split_sem, split_sem_bytes, total;
 };
 
 int validate(const sa_config* c, std::string* why) {
@@ -49,6 +50,8 @@ int validate(const sa_config* c, std::string* why) {
     return fail(SA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
   if (c->frames_per_chunk < 1 || c->tok_h < 1 || c->tok_w < 1)
     return fail(SA_ERR_INVALID_ARG, "frames_per_chunk, tok_h, tok_w must be >= 1");
+  if (c->frames_per_chunk > 1023 || c->tok_h > 2047 || c->tok_w > 2047)
+    return fail(SA_ERR_UNSUPPORTED, "frames_per_chunk must be < 1024 and tok_h, tok_w < 2048");
   if (c->sink_chunks < 0 || c->window_chunks < 1)
     return fail(SA_ERR_INVALID_ARG, "need sink_chunks >= 0 and window_chunks >= 1");
   if (c->sink_chunks + c->window_chunks > SA_MAX_ATTENDED)
@@ -100,6 +103,15 @@ Derived derive(const sa_config& c) {
   }
   d.off_kcur = off;
   off += align_up(d.chunk_elems * sizeof(__nv_bfloat16), 1024);
+  // split-tail scratch: partial rows, their lse, per-row merge counters
+  const size_t split_rows = static_cast<size_t>(sa::kMaxSplitSlots) * 2 * 2 * 128;
+  d.off_split_o = off;
+  off += align_up(split_rows * d.D * sizeof(float), 1024);
+  d.off_split_lse = off;
+  off += align_up(split_rows * sizeof(float), 1024);
+  d.off_split_sem = off;
+  d.split_sem_bytes = static_cast<size_t>(sa::kMaxSplitSlots) * 2 * 128 * sizeof(int);
+  off += align_up(d.split_sem_bytes, 1024);
   d.total = off;
   return d;
 }
@@ -171,6 +183,47 @@ bool encode_blhd(CUtensorMap* map, const void* base, const Derived& d) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Persistent grid: one CTA per SM at most; with the split tail allowed, a problem
+// of fewer work tiles than SMs gets two CTAs per tile (key-range halves).
+unsigned attend_grid(const Derived& d, int sm_count, bool split_ok) {
+  const int n_qt = (d.L + 127) / 128;
+  const long long n_work = 1LL * d.B * d.H * ((n_qt + 1) / 2);
+  long long g = n_work < sm_count ? n_work : sm_count;
+  if (split_ok && n_work < sm_count) g = 2 * n_work < sm_count ? 2 * n_work : sm_count;
+  return static_cast<unsigned>(g);
+}
+
+// The attention kernel instantiations: head dim 128 / 64, dense / block-sparse.
+template <int D, bool kSparse>
+void launch_attend_tc_t(unsigned grid, cudaStream_t s, const CUtensorMap& a, const CUtensorMap& b,
+                        const CUtensorMap& c, const AttendParams& ap) {
+  sa::attend_tc_kernel<D, kSparse>
+      <<<grid, sa::TcShape<D>::kThreads, sa::TcShape<D>::kSmemBytes, s>>>(a, b, c, ap);
+}
+
+void launch_attend_tc(int D, bool sparse, unsigned grid, cudaStream_t s, const CUtensorMap& a,
+                      const CUtensorMap& b, const CUtensorMap& c, const AttendParams& ap) {
+  if (D == 128)
+    sparse ? launch_attend_tc_t<128, true>(grid, s, a, b, c, ap)
+           : launch_attend_tc_t<128, false>(grid, s, a, b, c, ap);
+  else
+    sparse ? launch_attend_tc_t<64, true>(grid, s, a, b, c, ap)
+           : launch_attend_tc_t<64, false>(grid, s, a, b, c, ap);
+}
+
+// Every instantiation: the register count the setmaxnreg split assumes, and the
+// dynamic shared memory it needs.
+template <int D, bool kSparse>
+bool prepare_attend_tc_t() {
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, sa::attend_tc_kernel<D, kSparse>) != cudaSuccess ||
+      fa.numRegs != sa::TcShape<D>::kLaunchRegs)
+    return false;
+  return cudaFuncSetAttribute(sa::attend_tc_kernel<D, kSparse>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              sa::TcShape<D>::kSmemBytes) == cudaSuccess;
+}
 
 __global__ void exp2_probe_kernel(const float* x, float* y, int n, int poly) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -271,7 +324,8 @@ int stage_keys(sa_handle* h, const void* Kc, sa_stream stream) {
 }
 
 int attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final, void* O,
-                  float* lse, sa_stream stream, bool simt) {
+                  float* lse, sa_stream stream, bool simt, bool debug_stall = false,
+                  const uint8_t* block_mask = nullptr) {
   int rc = check_handle(h);
   if (rc != SA_OK) return rc;
   if (Q == nullptr || Vc == nullptr || O == nullptr)
@@ -317,6 +371,12 @@ int attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final
   ap.scale_log2 = d.scale * 1.4426950408889634f;
   ap.rope = h->rope();
   ap.status = h->status();
+  ap.debug_stall_producer = debug_stall ? 1 : 0;
+  ap.block_mask = block_mask;
+  ap.split_o = reinterpret_cast<float*>(h->buf + d.off_split_o);
+  ap.split_lse = reinterpret_cast<float*>(h->buf + d.off_split_lse);
+  ap.split_sem = reinterpret_cast<int*>(h->buf + d.off_split_sem);
+  ap.split_ok = h->sm_count <= 2 * sa::kMaxSplitSlots ? 1 : 0;
 
   if (simt) {
     const long long rows = 1LL * d.B * d.H * d.L;
@@ -329,15 +389,8 @@ int attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final
     CUtensorMap tm_v;
     if (!encode_blhd(&tm_v, Vc, d)) return h->fail(SA_ERR_CUDA, "TMA descriptor for Vc failed");
     const CUtensorMap& tm_cache = h->has_cache ? h->tm_tier[tier] : h->tm_kcur;
-    const int n_qt = (d.L + 127) / 128;
-    const long long n_work = 1LL * d.B * d.H * ((n_qt + 1) / 2);
-    const unsigned grid = static_cast<unsigned>(n_work < h->sm_count ? n_work : h->sm_count);
-    if (d.D == 128)
-      sa::attend_tc_kernel<128><<<grid, sa::TcShape<128>::kThreads, sa::TcShape<128>::kSmemBytes,
-                                  s>>>(tm_cache, h->tm_kcur, tm_v, ap);
-    else
-      sa::attend_tc_kernel<64><<<grid, sa::TcShape<64>::kThreads, sa::TcShape<64>::kSmemBytes,
-                                 s>>>(tm_cache, h->tm_kcur, tm_v, ap);
+    launch_attend_tc(d.D, block_mask != nullptr, attend_grid(d, h->sm_count, ap.split_ok != 0), s,
+                     tm_cache, h->tm_kcur, tm_v, ap);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
@@ -450,15 +503,9 @@ int attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc, 
   rc = launch_rope_transpose(h, Kc, nullptr, keys, nullptr, s);
   if (rc != SA_OK) return rc;
   const CUtensorMap& tm_cache = h->has_cache ? h->tm_tier[tier] : tm_keys;
-  const int n_qt = (d.L + 127) / 128;
-  const long long n_work = 1LL * d.B * d.H * ((n_qt + 1) / 2);
-  const unsigned grid = static_cast<unsigned>(n_work < h->sm_count ? n_work : h->sm_count);
-  if (d.D == 128)
-    sa::attend_tc_kernel<128><<<grid, sa::TcShape<128>::kThreads, sa::TcShape<128>::kSmemBytes,
-                                s>>>(tm_cache, tm_keys, tm_v, ap);
-  else
-    sa::attend_tc_kernel<64><<<grid, sa::TcShape<64>::kThreads, sa::TcShape<64>::kSmemBytes,
-                               s>>>(tm_cache, tm_keys, tm_v, ap);
+  ap.split_ok = 0;  // no scratch but the fixed key array: no split tail
+  launch_attend_tc(d.D, false, attend_grid(d, h->sm_count, false), s, tm_cache, tm_keys, tm_v,
+                   ap);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
     return h->fail(SA_ERR_CUDA, std::string("attend launch: ") + cudaGetErrorString(e));
@@ -546,7 +593,8 @@ SA_API int sa_create(const sa_config* cfg, void* dev_buf, size_t bytes, sa_handl
   fill(t, (d.S + d.W) * d.F, d.dt2);
   fill(th, d.th, d.dh2);
   fill(tw, d.tw, d.dw2);
-  bool ok = cudaMemset(h->buf + d.off_status, 0, 1024) == cudaSuccess;
+  bool ok = cudaMemset(h->buf + d.off_status, 0, 1024) == cudaSuccess &&
+            cudaMemset(h->buf + d.off_split_sem, 0, d.split_sem_bytes) == cudaSuccess;
   ok = ok && cudaMemcpy(h->buf + d.off_rope_t, t.data(), t.size() * sizeof(float2),
                         cudaMemcpyHostToDevice) == cudaSuccess;
   ok = ok && cudaMemcpy(h->buf + d.off_rope_h, th.data(), th.size() * sizeof(float2),
@@ -574,25 +622,11 @@ SA_API int sa_create(const sa_config* cfg, void* dev_buf, size_t bytes, sa_handl
   }
   // The kernel's register split assumes it is launched with exactly
   // TcShape::kLaunchRegs registers per thread; refuse to run otherwise.
-  cudaFuncAttributes fa128, fa64;
-  if (cudaFuncGetAttributes(&fa128, sa::attend_tc_kernel<128>) != cudaSuccess ||
-      cudaFuncGetAttributes(&fa64, sa::attend_tc_kernel<64>) != cudaSuccess ||
-      fa128.numRegs != sa::TcShape<128>::kLaunchRegs ||
-      fa64.numRegs != sa::TcShape<64>::kLaunchRegs) {
-    g_error = "attention kernel built with an unexpected register count";
+  if (!prepare_attend_tc_t<128, false>() || !prepare_attend_tc_t<128, true>() ||
+      !prepare_attend_tc_t<64, false>() || !prepare_attend_tc_t<64, true>()) {
+    g_error = "attention kernel: unexpected register count or shared memory attribute failed";
     delete h;
     return SA_ERR_UNSUPPORTED;
-  }
-  cudaError_t e = cudaFuncSetAttribute(sa::attend_tc_kernel<128>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       sa::TcShape<128>::kSmemBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(sa::attend_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             sa::TcShape<64>::kSmemBytes);
-  if (e != cudaSuccess) {
-    g_error = std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e);
-    delete h;
-    return SA_ERR_CUDA;
   }
   *out = h;
   return SA_OK;
@@ -613,6 +647,7 @@ SA_API int sa_reset(sa_handle* h) {
   h->count[0] = h->count[1] = 0;
   h->staged_chunk = -1;
   if (cudaMemset(h->buf + h->d.off_status, 0, 1024) != cudaSuccess ||
+      cudaMemset(h->buf + h->d.off_split_sem, 0, h->d.split_sem_bytes) != cudaSuccess ||
       cudaDeviceSynchronize() != cudaSuccess)
     return h->fail(SA_ERR_CUDA, "clearing the status word failed");
   return SA_OK;
@@ -667,6 +702,45 @@ SA_API int sa_debug_attend_simt(sa_handle* h, const void* Q, const void* Kc, con
 SA_API int sa_attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
                              int step_is_final, void* O, float* lse, sa_stream stream) {
   return attend_noalloc(h, Q, Kc, Vc, step_is_final, O, lse, stream);
+}
+
+SA_API int sa_attend_sparse(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
+                            int step_is_final, const uint8_t* block_mask, void* O, float* lse,
+                            sa_stream stream) {
+  int rc = check_handle(h);
+  if (rc != SA_OK) return rc;
+  if (block_mask == nullptr) return h->fail(SA_ERR_INVALID_ARG, "block_mask must be non-NULL");
+  if (Q == nullptr || Kc == nullptr || Vc == nullptr || O == nullptr)
+    return h->fail(SA_ERR_INVALID_ARG, "Q, Kc, Vc and O must be non-NULL");
+  if (!aligned16(Q) || !aligned16(Vc) || !aligned16(O) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 || O == Q || O == Vc || O == Kc)
+    return h->fail(SA_ERR_INVALID_ARG, "Q, Vc, O must be 16-byte aligned, lse 4-byte aligned, "
+                                       "O must not alias an input");
+  rc = stage_keys(h, Kc, stream);
+  if (rc != SA_OK) return rc;
+  return attend_staged(h, Q, Vc, step_is_final, O, lse, stream, false, false, block_mask);
+}
+
+SA_API int sa_block_grid(const sa_config* cfg, int32_t chunk, int32_t* n_q_tiles,
+                         int32_t* n_k_tiles) {
+  std::string why;
+  if (validate(cfg, &why) != SA_OK || chunk < 0 || n_q_tiles == nullptr || n_k_tiles == nullptr) {
+    g_error = why.empty() ? "bad chunk or NULL output" : why;
+    return SA_ERR_INVALID_ARG;
+  }
+  const Derived d = derive(*cfg);
+  int ids[SA_MAX_ATTENDED];
+  const int n = plan_ids(d, chunk, ids);
+  *n_q_tiles = (d.L + 127) / 128;
+  *n_k_tiles = n * ((d.L + 127) / 128);
+  return SA_OK;
+}
+
+SA_API int sa_debug_attend_stalled(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
+                                   int step_is_final, void* O, sa_stream stream) {
+  int rc = stage_keys(h, Kc, stream);
+  if (rc != SA_OK) return rc;
+  return attend_staged(h, Q, Vc, step_is_final, O, nullptr, stream, false, true);
 }
 
 SA_API int sa_debug_exp2(int use_polynomial, const float* x, float* y, int n, sa_stream stream) {

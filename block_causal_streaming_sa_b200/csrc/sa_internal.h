@@ -10,6 +10,7 @@
 namespace sa {
 
 constexpr int kMaxGroups = SA_MAX_ATTENDED;
+constexpr int kMaxSplitSlots = 128;  // tail tiles that may be split (grids of up to 256 CTAs)
 
 // Device status word bits (written with atomicOr, read by sa_get_status).
 constexpr unsigned kDevErrTimeout = 1u;
@@ -59,6 +60,18 @@ struct AttendParams {
   float scale_log2;  // softmax scale * log2(e)
   RopeTables rope;
   unsigned* status;
+  const uint8_t* block_mask;  // optional [B][H][n_q_tiles][n_k_tiles]: nonzero = the 128x128
+                              // block is attended; null = dense
+  // Split tail: when the last round of work tiles would leave most CTAs idle,
+  // its tiles are split into two key-range halves; each half writes a
+  // normalised fp32 partial row and its lse, and per row the second finisher
+  // (atomic counter) merges both. Regions sized for kMaxSplitSlots tiles.
+  float* split_o;    // [slot][query tile 0/1][half][128 rows][D]
+  float* split_lse;  // [slot][query tile][half][128 rows]
+  int* split_sem;    // [slot][query tile][128 rows], zero between launches
+  int split_ok;
+  int debug_stall_producer;  // test hook: 1 = the TMA producer issues nothing, so the
+                             // MMA warp's bounded wait runs out (timeout path)
 };
 
 }  // namespace sa

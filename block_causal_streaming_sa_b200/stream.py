@@ -65,6 +65,22 @@ class StreamingAttention:
            step_is_final, self._ptr(out, "O"), lse_ptr, self._stream(stream))
         return out
 
+    def attend_sparse(self, Q, Kc, Vc, step_is_final, block_mask, out=None, lse=None,
+                      stream=None):
+        """Block-sparse attention; block_mask: uint8 [B, H, n_q_tiles, n_k_tiles] on the device."""
+        b, l, h, _ = self.shape
+        nq, nk = B.sa_block_grid(self.cfg, self.chunk_count(B.SA_TIER_NOISY))
+        if block_mask.dtype != torch.uint8 or tuple(block_mask.shape) != (b, h, nq, nk) \
+                or not block_mask.is_contiguous() or block_mask.device != self.device:
+            raise ValueError(f"block_mask must be contiguous uint8 {(b, h, nq, nk)} on {self.device}")
+        if out is None:
+            out = torch.empty(self.shape, dtype=torch.bfloat16, device=self.device)
+        lse_ptr = 0 if lse is None else lse.data_ptr()
+        B.sa_attend_sparse(self.handle, self._ptr(Q, "Q"), self._ptr(Kc, "Kc"), self._ptr(Vc, "Vc"),
+                           step_is_final, block_mask.data_ptr(), self._ptr(out, "O"), lse_ptr,
+                           self._stream(stream))
+        return out
+
     def reset(self):
         B.sa_reset(self.handle)
 

@@ -136,6 +136,25 @@ SA_API int sa_append_chunk(sa_handle* h, int tier, const void* K, const void* V,
 SA_API int sa_attend(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
                      int step_is_final, void* O, float* lse, sa_stream stream);
 
+/* Block-sparse attention ("Vidu S2 vs PixVerse R2：实时视频的两条技术路线", section
+ * 选择四：速度从哪里来: PixVerse R2 learns block-sparse attention and skips more than
+ * 90 % of the blocks). Same as sa_attend, but only the blocks flagged in
+ * block_mask are attended: a block is 128 query rows (tile qt: rows 128*qt ..)
+ * x 128 keys of the attended key sequence (the attended chunks in ascending id
+ * order, each cut into 128-key tiles from its first token, the last tile of a
+ * chunk possibly short). block_mask: device uint8 [B][H][n_q_tiles][n_k_tiles]
+ * (nonzero = attended), from sa_block_grid for the current chunk; read only.
+ * Key tiles no query tile of a 256-row pair needs are neither loaded nor
+ * multiplied. A row that sees no key gets O = 0 and lse = -inf. */
+SA_API int sa_attend_sparse(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
+                            int step_is_final, const uint8_t* block_mask, void* O, float* lse,
+                            sa_stream stream);
+
+/* Block grid of chunk `chunk`'s attention for config cfg: *n_q_tiles =
+ * ceil(L / 128), *n_k_tiles = (attended chunks) * ceil(L / 128). Host only. */
+SA_API int sa_block_grid(const sa_config* cfg, int32_t chunk, int32_t* n_q_tiles,
+                         int32_t* n_k_tiles);
+
 /* The two halves of sa_attend, for callers that time or schedule them apart.
  * sa_stage_keys rotates the generating chunk's Kc ([B, L, H, D] bf16) by its
  * in-chunk positions into the handle's key scratch (one HBM-bound kernel).
@@ -175,6 +194,14 @@ SA_API int sa_attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const 
  * kernel, an order of magnitude slower; not used by sa_attend. */
 SA_API int sa_debug_attend_simt(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
                                 int step_is_final, void* O, float* lse, sa_stream stream);
+
+/* Test hook for the failure path: runs sa_attend with the kernel's TMA producer
+ * switched off, so the MMA warp's wait for the first key tile runs out (about
+ * one second). The kernel then drains, frees its tensor memory and sets the
+ * device status word: sa_get_status returns SA_ERR_TIMEOUT until sa_reset. O is
+ * left unspecified. The CUDA context stays usable. */
+SA_API int sa_debug_attend_stalled(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
+                                   int step_is_final, void* O, sa_stream stream);
 
 /* Evaluate the attention kernel's device exponentials on n fp32 values (device
  * pointers x, y): use_polynomial = 0 -> the exp unit (ex2.approx), 1 -> the

@@ -93,6 +93,24 @@ class Pair:
                                           final, rows=rows_idx)
         return o_gpu, o_ref, l_gpu, l_ref
 
+    def attend_sparse(self, step, final, block_mask, rows=None, tensors=None):
+        """Block-sparse attention on both sides; block_mask: numpy uint8 [B, H, nq, nk]."""
+        from oracle.sparse import block_sparse_attend
+
+        Q, Kc, Vc = tensors if tensors is not None else self.tensors(("Q", "Kc", "Vc"), step)
+        b, l, h, _ = Q.shape
+        lse = torch.empty((b, h, l), dtype=torch.float32, device="cuda")
+        mask = torch.from_numpy(np.ascontiguousarray(block_mask)).cuda()
+        out = self.gpu.attend_sparse(Q.cuda(), Kc.cuda(), Vc.cuda(), final, mask, lse=lse)
+        torch.cuda.synchronize()
+        rows_idx = np.arange(l) if rows is None else np.asarray(rows)
+        o_gpu = f64(out.cpu())[self.bsel][:, rows_idx][:, :, self.hsel]
+        l_gpu = lse.cpu().double().numpy()[self.bsel][:, self.hsel][:, :, rows_idx]
+        sub = block_mask[self.bsel][:, self.hsel]
+        o_ref, l_ref = block_sparse_attend(self.oracle, self._slice(Q), self._slice(Kc),
+                                           self._slice(Vc), final, sub, rows=rows_idx)
+        return o_gpu, o_ref, l_gpu, l_ref
+
     def check_layout(self):
         for tier in (NOISY, CLEAN):
             got = self.gpu.layout(tier)

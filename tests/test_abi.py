@@ -101,3 +101,17 @@ def test_null_handle_calls_fail_cleanly():
     assert lib.sa_chunk_count(None, 0) < 0
     assert lib.sa_destroy(None) == sa.SA_OK
     assert sa.last_error() != ""
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_block_grid_matches_oracle_tiling(name):
+    from oracle.sparse import key_tiles
+
+    w = WORKLOADS[name]
+    cfg = sa.make_config(**w.config_dict())
+    model = RingCacheModel(w.sink, w.window)
+    for c in range(12):
+        nq, nk = sa.sa_block_grid(cfg, c)
+        assert nq == -(-w.chunk_len // 128)
+        assert nk == len(key_tiles([w.chunk_len] * len(model.attended())))
+        model.append()

@@ -1,0 +1,76 @@
+"""The multi-rank host path of bench.py on CPU: two gloo ranks.
+
+bench.py under torchrun runs one independent stream per rank (weak scaling);
+its only collectives are a barrier around the timed region and a max over
+ranks of each reported time. These tests drive that exact code (bench.Ranks,
+bench.whole_job_tflops) with world size 2 on the gloo backend, and check that
+the reference arm does its work on rank 0 only.
+"""
+
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      LOCAL_RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import bench
+
+    ranks = bench.Ranks("gloo", "cpu", timeout_s=60)
+    ranks.barrier()
+    local_ms = 10.0 * (rank + 1)          # rank 1 is the slow one
+    ms_max = ranks.max(local_ms)
+    value = bench.whole_job_tflops(2e12, ms_max, ranks.world)
+    ranks.barrier()
+    ranks.close()
+    out.put((rank, ms_max, value))
+
+
+def test_two_rank_barrier_max_and_weak_scaling_value():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    # both ranks see the slowest rank's time; value = work of both ranks / that time
+    assert [r[1] for r in res] == [20.0, 20.0]
+    assert res[0][2] == pytest.approx(2 * 2e12 / 20e-3 / 1e12)
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "0"], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_reference_arm_line_on_rank_zero():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny",
+                        "--steps", "2", "--warmup", "1"], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
