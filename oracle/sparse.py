@@ -17,6 +17,9 @@ from .attention import softmax_attention
 from .rope import rotate, token_positions
 from .stream import CLEAN, NOISY
 
+# (The reference image, when set, is not part of the block grid: reading R11
+# covers the chunks' keys only; block_sparse_attend requires no reference.)
+
 TILE = 128
 
 
@@ -36,14 +39,18 @@ def block_sparse_attend(orc, Q, Kc, Vc, final, block_mask, rows=None, heads=None
     cfg = orc.cfg
     c = orc.current_chunk()
     tier = CLEAN if final else NOISY
-    ids, rank = orc.attended(final)
-    L, F = cfg.chunk_len, cfg.frames
+    if orc.reference is not None:
+        raise ValueError("block-sparse attention takes no reference image")
+    Q, Kc, Vc = (np.asarray(t, dtype=np.float64) for t in (Q, Kc, Vc))
+    ids, base = orc.positions(final, orc.frames(Q))
+    L = Q.shape[1]
     rows = np.arange(L) if rows is None else np.asarray(rows)
     heads = range(cfg.heads) if heads is None else heads
     batches = range(cfg.batch) if batches is None else batches
     f, y, x = token_positions(L, cfg.tok_h, cfg.tok_w)
-    tiles = key_tiles([L] * len(ids))
-    Q, Kc, Vc = (np.asarray(t, dtype=np.float64) for t in (Q, Kc, Vc))
+    lengths = [L if j == c else orc.store[tier][j][0].shape[1] for j in ids]
+    starts = np.concatenate([[0], np.cumsum(lengths)])
+    tiles = key_tiles(lengths)
 
     O = np.zeros((len(batches), len(rows), len(heads), cfg.head_dim))
     lse = np.full((len(batches), len(heads), len(rows)), -np.inf)
@@ -52,16 +59,17 @@ def block_sparse_attend(orc, Q, Kc, Vc, final, block_mask, rows=None, heads=None
             keys, vals = [], []
             for j in ids:
                 Kj, Vj = (Kc, Vc) if j == c else orc.store[tier][j]
-                keys.append(rotate(Kj[b, :, h, :], rank[j] * F + f, y, x, cfg.theta))
+                fj, yj, xj = token_positions(Kj.shape[1], cfg.tok_h, cfg.tok_w)
+                keys.append(rotate(Kj[b, :, h, :], base[j] + fj, yj, xj, cfg.theta))
                 vals.append(Vj[b, :, h, :])
             keys, vals = np.concatenate(keys), np.concatenate(vals)
-            q = rotate(Q[b, rows, h, :], rank[c] * F + f[rows], y[rows], x[rows], cfg.theta)
+            q = rotate(Q[b, rows, h, :], base[c] + f[rows], y[rows], x[rows], cfg.theta)
             # visible keys of each query row: the keys of the flagged blocks of its tile
             mask = np.zeros((len(rows), len(keys)), dtype=bool)
             for ri, r in enumerate(rows):
                 for kt, (g, s, e) in enumerate(tiles):
                     if block_mask[b, h, r // TILE, kt]:
-                        mask[ri, g * L + s:g * L + e] = True
+                        mask[ri, starts[g] + s:starts[g] + e] = True
             seen = mask.any(axis=1)
             if seen.any():
                 o, l = softmax_attention(q[seen], keys, vals, cfg.softmax_scale, mask=mask[seen])

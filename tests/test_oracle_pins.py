@@ -420,14 +420,14 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     #    the masked full-stream pin
     c = orc.current_chunk()
     ref, _ = masked_full_attention(cfg, orc.history, c, Q, Kc, Vc, True)
-    real_attended = StreamOracle.attended
+    real_positions = StreamOracle.positions
 
-    def shifted_attended(self, final):
-        ids, ranks = real_attended(self, final)
-        ranks = dict(ranks)
-        ranks[ids[-1]] += 1
-        return ids, ranks
-    monkeypatch.setattr(StreamOracle, "attended", shifted_attended)
+    def shifted_positions(self, final, current_frames):
+        ids, base = real_positions(self, final, current_frames)
+        base = dict(base)
+        base[ids[-1]] += cfg.frames  # current chunk one chunk further away
+        return ids, base
+    monkeypatch.setattr(StreamOracle, "positions", shifted_positions)
     bad, _ = orc.attend(Q, Kc, Vc, True)
     monkeypatch.undo()
     assert np.abs(bad - ref).max() > 1e-3
