@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--sparsity", type=float, default=0.0,
                     help="block-sparse mode: share of 128x128 blocks skipped (seeded random mask)")
+    ap.add_argument("--ref-frames", type=int, default=0,
+                    help="frames of a reference image every chunk also attends (0: none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
@@ -295,6 +297,7 @@ def run_ours(args, w):
     import torch
 
     import block_causal_streaming_sa_b200 as sa
+    from sa_inputs import normal_bf16, seed_of
 
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
@@ -314,10 +317,22 @@ def run_ours(args, w):
     out_host = torch.empty(w.shape(), dtype=torch.bfloat16).pin_memory()
 
     # One handle (its own two-tier cache) per attention layer of the workload.
-    layers = [sa.StreamingAttention(w.config_dict(), device=dev) for _ in range(w.layers)]
+    cfg = dict(w.config_dict(), ref_frames=args.ref_frames)
+    layers = [sa.StreamingAttention(cfg, device=dev) for _ in range(w.layers)]
     attn = layers[0]
     sp = stream.cuda_stream
     flops = attend_flops(w)
+    ref_len = args.ref_frames * w.tok_h * w.tok_w
+    if args.ref_frames > 0:
+        # A reference image of ref_frames frames, set once (its keys are rotated
+        # on the way in); every attention also reads its ref_len keys.
+        ref_shape = (w.batch, ref_len, w.heads, w.head_dim)
+        Kref, Vref = (normal_bf16(seed_of(w.name, "reference", n), ref_shape).to(dev)
+                      for n in ("K", "V"))
+        for layer in layers:
+            layer.set_reference(Kref, Vref)
+        torch.cuda.synchronize(dev)
+        flops += 4.0 * w.batch * w.heads * w.chunk_len * ref_len * w.head_dim
     steps_per_chunk = w.steps
     attends_per_chunk = steps_per_chunk * w.layers
     appends_per_chunk = 2 * w.layers
@@ -469,6 +484,7 @@ def run_ours(args, w):
                   f"read per attention vs {L2_BYTES / 2**20:.0f} MiB L2",
             "parallelism": f"replicas{world}" if world > 1 else "single",
             "block_sparsity": args.sparsity,
+            "ref_frames": args.ref_frames, "ref_tokens": ref_len,
         },
         "roofline": {
             "bound": "tensor",

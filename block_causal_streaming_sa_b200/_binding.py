@@ -38,6 +38,7 @@ class SaConfig(ctypes.Structure):
         ("window_chunks", ctypes.c_int32),
         ("softmax_scale", ctypes.c_float),
         ("rope_theta", ctypes.c_float),
+        ("ref_frames", ctypes.c_int32),
     ]
 
 
@@ -60,8 +61,12 @@ _SIGNATURES = {
     "sa_destroy": (_I, [_P]),
     "sa_reset": (_I, [_P]),
     "sa_append_chunk": (_I, [_P, _I, _P, _P, _P]),
+    "sa_append_chunk_frames": (_I, [_P, _I, _P, _P, _I, _P]),
+    "sa_set_reference": (_I, [_P, _P, _P, _P]),
     "sa_attend": (_I, [_P, _P, _P, _P, _I, _P, _P, _P]),
+    "sa_attend_frames": (_I, [_P, _P, _P, _P, _I, _I, _P, _P, _P]),
     "sa_stage_keys": (_I, [_P, _P, _P]),
+    "sa_stage_keys_frames": (_I, [_P, _P, _I, _P]),
     "sa_attend_staged": (_I, [_P, _P, _P, _I, _P, _P, _P]),
     "sa_debug_attend_simt": (_I, [_P, _P, _P, _P, _I, _P, _P, _P]),
     "sa_attend_noalloc": (_I, [_P, _P, _P, _P, _I, _P, _P, _P]),
@@ -72,6 +77,7 @@ _SIGNATURES = {
     "sa_chunk_count": (_I, [_P, _I]),
     "sa_debug_layout": (_I, [_P, _I, _I32P, _I]),
     "sa_plan": (_I, [_CFGP, ctypes.c_int32, _I32P, _I32P, _I32P, _I]),
+    "sa_stream_plan": (_I, [_P, _I, _I, _I32P, _I32P, _I32P, _I]),
     "sa_slot_of": (_I, [_CFGP, ctypes.c_int32]),
     "sa_get_status": (_I, [_P, _P]),
     "sa_last_error": (ctypes.c_char_p, [_P]),
@@ -115,9 +121,9 @@ def _check(status, handle=None):
 
 
 def make_config(batch, heads, head_dim, frames_per_chunk, tok_h, tok_w, sink_chunks,
-                window_chunks, softmax_scale=0.0, rope_theta=0.0):
+                window_chunks, softmax_scale=0.0, rope_theta=0.0, ref_frames=0):
     return SaConfig(batch, heads, head_dim, frames_per_chunk, tok_h, tok_w, sink_chunks,
-                    window_chunks, softmax_scale, rope_theta)
+                    window_chunks, softmax_scale, rope_theta, ref_frames)
 
 
 def sa_validate_config(cfg):
@@ -144,6 +150,26 @@ def sa_reset(handle):
 
 def sa_append_chunk(handle, tier, K, V, stream=0):
     _check(lib().sa_append_chunk(handle, tier, _P(K), _P(V), _P(stream)), handle)
+
+
+def sa_append_chunk_frames(handle, tier, K, V, n_frames, stream=0):
+    _check(lib().sa_append_chunk_frames(handle, tier, _P(K), _P(V), int(n_frames), _P(stream)),
+           handle)
+
+
+def sa_set_reference(handle, K, V, stream=0):
+    """Set / replace the reference image (K = V = 0 clears it)."""
+    _check(lib().sa_set_reference(handle, _P(K or None), _P(V or None), _P(stream)), handle)
+
+
+def sa_attend_frames(handle, Q, Kc, Vc, n_frames, step_is_final, O, lse=0, stream=0):
+    _check(lib().sa_attend_frames(handle, _P(Q), _P(Kc), _P(Vc), int(n_frames),
+                                  int(bool(step_is_final)), _P(O), _P(lse or None), _P(stream)),
+           handle)
+
+
+def sa_stage_keys_frames(handle, Kc, n_frames, stream=0):
+    _check(lib().sa_stage_keys_frames(handle, _P(Kc), int(n_frames), _P(stream)), handle)
 
 
 def sa_attend(handle, Q, Kc, Vc, step_is_final, O, lse=0, stream=0):
@@ -212,6 +238,17 @@ def sa_plan(cfg, chunk):
     if n < 0:
         raise SaError(-n, last_error())
     return list(ids[:n]), list(slots[:n]), list(tb[:n])
+
+
+def sa_stream_plan(handle, step_is_final, n_frames):
+    """(ids, t_base, lens) of the plan the handle would run now for a generating
+    chunk of n_frames frames (the reference image is not listed)."""
+    cap = SA_MAX_ATTENDED
+    ids, tb, lens = ((ctypes.c_int32 * cap)() for _ in range(3))
+    n = lib().sa_stream_plan(handle, int(bool(step_is_final)), int(n_frames), ids, tb, lens, cap)
+    if n < 0:
+        raise SaError(-n, last_error(handle))
+    return list(ids[:n]), list(tb[:n]), list(lens[:n])
 
 
 def sa_slot_of(cfg, chunk):

@@ -1,6 +1,6 @@
-// Plain fp32 SIMT attention over the sink + window chunks: one warp per query
-// row, lanes split the head dimension, exact exp2f, online softmax over keys in
-// ascending chunk order. Reads the same cache layout as the tensor-core kernel
+// Plain fp32 SIMT attention over the reference image (if set) and the sink +
+// window chunks: one warp per query row, lanes split the head dimension, exact
+// exp2f, online softmax over the key groups in order. Reads the same cache layout as the tensor-core kernel
 // and applies the same query-side relocated rotation (rounded to fp16 like the
 // MMA operand), so it is an independent check of the tensor-core machinery.
 // Debug path only: sa_debug_attend_simt.
@@ -37,7 +37,8 @@ __global__ void __launch_bounds__(256) attend_simt_kernel(AttendParams p) {
 #pragma unroll
   for (int d = 0; d < DPL; ++d) acc[d] = 0.f;
 
-  const size_t plane = static_cast<size_t>(p.L) * D;
+  const size_t plane = static_cast<size_t>(p.L_plane) * D;
+  const size_t ref_plane = static_cast<size_t>(p.L_ref) * D;
   for (int g = 0; g < p.n_groups; ++g) {
     const AttendGroup grp = p.groups[g];
     float q[DPL];
@@ -53,6 +54,10 @@ __global__ void __launch_bounds__(256) attend_simt_kernel(AttendParams p) {
     if (grp.src == 0) {
       kb = p.cache + ((static_cast<size_t>(grp.slot) * 2 * p.B + b) * p.H + h) * plane;
       vb = p.cache + (((static_cast<size_t>(grp.slot) * 2 + 1) * p.B + b) * p.H + h) * plane;
+      vstride = D;
+    } else if (grp.src == 2) {
+      kb = p.ref + (static_cast<size_t>(b) * p.H + h) * ref_plane;
+      vb = p.ref + ((static_cast<size_t>(p.B) + b) * p.H + h) * ref_plane;
       vstride = D;
     } else {
       kb = p.k_cur + (static_cast<size_t>(b) * p.H + h) * plane;

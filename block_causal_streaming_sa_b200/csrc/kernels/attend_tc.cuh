@@ -2,18 +2,20 @@
 //
 // What it computes ("Vidu S2 vs PixVerse R2：实时视频的两条技术路线", sections
 // 「实时」改变了什么 and 选择三：有上限的记忆): for every query row of the chunk
-// being generated, softmax attention over the keys of the cached sink and window
-// chunks of one TwinCache tier plus the chunk's own keys, with the temporal RoPE
-// position of chunk j relocated to rank(j) * F. With kSparse, only the 128 x 128
-// blocks a caller flags are attended (section 选择四：速度从哪里来: block-sparse
-// attention with most blocks skipped).
+// being generated, softmax attention over the keys of the reference image (if
+// set: "Vidu S2：实时可交互、可编辑、可立体的视频生成", section 2.2), the cached sink and
+// window chunks of one TwinCache tier and the chunk's own keys, with the
+// temporal RoPE base of chunk j relocated to ref_frames + the frames of the
+// attended chunks before it (rank(j) * F when all have F frames). With
+// kSparse, only the 128 x 128 blocks a caller flags are attended (section
+// 选择四：速度从哪里来: block-sparse attention with most blocks skipped).
 //
 // Design (B200):
 //  * persistent CTAs, one per SM; a work tile is two 128-row query tiles of one
 //    (batch, head), so every K/V tile brought in by TMA feeds two MMAs;
 //  * warp 0 (one lane): TMA producer over a ring of NSTAGE 128x D tiles,
-//    K_0 V_0 K_1 V_1 ..., 128-byte swizzle, straight from the cache slots and
-//    from the caller's V (no gather copy);
+//    K_0 V_0 K_1 V_1 ..., 128-byte swizzle, straight from the cache slots, the
+//    reference planes and the caller's V (no gather copy);
 //  * warp 1 (one lane): tcgen05.mma issuer. S_i = Q_i K^T (SS form, fp16, both
 //    operands K-major in shared memory) into TMEM, then O_i += P_i V (TS form,
 //    bf16: P_i read from TMEM, written over the upper half of S_i, V MN-major
@@ -33,7 +35,7 @@
 //    stays in registers without spills; the epilogue is a separate function so
 //    its registers do not add to the score loop's;
 //  * RoPE: keys are stored rotated by their in-chunk position; the relocated
-//    temporal base rank(j) * F of the attended chunk is applied by re-turning
+//    temporal base of the attended chunk is applied by re-turning
 //    the temporal band of the query tile when the key stream moves to the next
 //    chunk, before the first QK^T MMA of that chunk;
 //  * work units: rounds of gridDim.x work tiles; when the last round holds at
@@ -224,6 +226,7 @@ __global__ void __launch_bounds__(384, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tm_cache,
                      const __grid_constant__ CUtensorMap tm_kcur,
                      const __grid_constant__ CUtensorMap tm_vcur,
+                     const __grid_constant__ CUtensorMap tm_ref,
                      const __grid_constant__ AttendParams p) {
   using T = TcShape<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -336,6 +339,7 @@ __global__ void __launch_bounds__(384, 1)
       ptx::tma_prefetch_desc(&tm_cache);
       ptx::tma_prefetch_desc(&tm_kcur);
       ptx::tma_prefetch_desc(&tm_vcur);
+      if (groups[0].src == 2) ptx::tma_prefetch_desc(&tm_ref);
       int stage = 0;
       uint32_t phase = 0, filled_mask = 0, filled_parity = 0;
       bool ok = true;
@@ -363,6 +367,9 @@ __global__ void __launch_bounds__(384, 1)
                 if (grp.src == 0) {
                   const int plane = ((grp.slot * 2 + kv) * p.B + b) * p.H + h;
                   ptx::tma_load_3d(dst + kb * T::kBox, &tm_cache, full, kb * 64, t * T::BN, plane);
+                } else if (grp.src == 2) {
+                  ptx::tma_load_3d(dst + kb * T::kBox, &tm_ref, full, kb * 64, t * T::BN,
+                                   (kv * p.B + b) * p.H + h);
                 } else if (kv == 0) {
                   ptx::tma_load_3d(dst + kb * T::kBox, &tm_kcur, full, kb * 64, t * T::BN,
                                    b * p.H + h);

@@ -4,12 +4,13 @@
 // each token's position in space and in time) is applied with the band
 // reading [t | h | w], pair (2i, 2i+1) of a band turned by pos * theta^(-2i/d).
 //
-// Keys enter the cache rotated by their IN-CHUNK position and stored as fp16 (frame f within the
-// chunk, row y, column x). The relocated temporal base of a cached chunk
-// ("RoPE relocation", section 选择三 of "Vidu S2 vs PixVerse R2") changes as the
-// window slides, so it is not baked in: a rotation by rank(j) * F of every key
-// of chunk j is, inside q . k, the same as turning q back by rank(j) * F, which
-// the attention kernels do once per attended chunk on the query side.
+// Keys enter the cache rotated by their IN-CHUNK position and stored as fp16
+// (frame f within the chunk, row y, column x). The relocated temporal base
+// base(j) of a cached chunk ("RoPE relocation", section 选择三 of "Vidu S2 vs
+// PixVerse R2") changes as the window slides, so it is not baked in: rotating
+// every key of chunk j by base(j) is, inside q . k, the same as turning q back by
+// base(j), so a query at base(c) + f is turned by base(c) - base(j) + f, once per
+// attended chunk, on the query side (the reference image has base 0).
 #pragma once
 
 #include <cstdint>
@@ -66,9 +67,9 @@ __device__ __forceinline__ void st_v4(void* p, uint4 v) {
 }
 
 // One block per token (b, l); thread t moves 16-byte chunk t % (D/8) of head
-// t / (D/8). blockIdx.y: 0 = K (bf16 in, rotated, fp16 out), 1 = V (bf16, copied). Loads are fully
-// coalesced (a token's H*D values are contiguous); each head's 2*D bytes are
-// stored contiguously into its [B, H, L, D] plane.
+// t / (D/8). blockIdx.y: 0 = K (bf16 in, rotated, fp16 out), 1 = V (bf16,
+// copied). Loads are fully coalesced (a token's H*D values are contiguous); each head's 2*D bytes are
+// stored contiguously into its [B, H, L_out, D] plane.
 __global__ void rope_transpose_kernel(AppendParams p) {
   const int vec_per_head = p.D >> 3;
   const int t = threadIdx.x;
@@ -81,7 +82,7 @@ __global__ void rope_transpose_kernel(AppendParams p) {
   const int b = tok / p.L, l = tok - b * p.L;
   const int h = t / vec_per_head, c = t - h * vec_per_head;
   const size_t src = (static_cast<size_t>(tok) * p.H + h) * p.D + c * 8;
-  const size_t dst = ((static_cast<size_t>(b) * p.H + h) * p.L + l) * p.D + c * 8;
+  const size_t dst = ((static_cast<size_t>(b) * p.H + h) * p.L_out + l) * p.D + c * 8;
   uint4 v = ld_nc_v4(in + src);
   if (!is_v) {
     const int f = l / p.rope.frame_tokens;

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -31,11 +32,13 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Derived {
   int B, H, D, F, th, tw, S, W, R, L;
+  int RF, Lref;  // reference image: frames, keys
   int dt2, dh2, dw2;
   float scale, theta;
   size_t chunk_elems;  // B * H * L * D
+  size_t ref_elems;    // B * H * Lref * D
   // byte offsets inside the device buffer
-  size_t off_status, off_rope_t, off_rope_h, off_rope_w, off_tier[2], off_kcur;
+  size_t off_status, off_rope_t, off_rope_h, off_rope_w, off_tier[2], off_kcur, off_ref;
   size_t off_split_o, off_split_lse, off_split_sem, split_sem_bytes, total;
 };
 
@@ -54,10 +57,18 @@ int validate(const sa_config* c, std::string* why) {
     return fail(SA_ERR_UNSUPPORTED, "frames_per_chunk must be < 1024 and tok_h, tok_w < 2048");
   if (c->sink_chunks < 0 || c->window_chunks < 1)
     return fail(SA_ERR_INVALID_ARG, "need sink_chunks >= 0 and window_chunks >= 1");
-  if (c->sink_chunks + c->window_chunks > SA_MAX_ATTENDED)
-    return fail(SA_ERR_UNSUPPORTED, "sink_chunks + window_chunks exceeds SA_MAX_ATTENDED");
+  if (c->ref_frames < 0 || c->ref_frames > 1023)
+    return fail(SA_ERR_INVALID_ARG, "ref_frames must be in 0..1023");
+  if (c->sink_chunks + c->window_chunks + (c->ref_frames > 0 ? 1 : 0) > SA_MAX_ATTENDED)
+    return fail(SA_ERR_UNSUPPORTED,
+                "sink_chunks + window_chunks (+ 1 with a reference) exceeds SA_MAX_ATTENDED");
   const long long L = 1LL * c->frames_per_chunk * c->tok_h * c->tok_w;
   if (L > SA_MAX_CHUNK_LEN) return fail(SA_ERR_UNSUPPORTED, "chunk longer than SA_MAX_CHUNK_LEN");
+  const long long Lref = 1LL * c->ref_frames * c->tok_h * c->tok_w;
+  if (Lref > SA_MAX_CHUNK_LEN)
+    return fail(SA_ERR_UNSUPPORTED, "reference longer than SA_MAX_CHUNK_LEN");
+  if (1LL * c->batch * Lref > (1LL << 31) - 1)
+    return fail(SA_ERR_UNSUPPORTED, "batch * reference too big");
   if (1LL * c->heads * c->head_dim / 8 > 1024)
     return fail(SA_ERR_UNSUPPORTED, "heads * head_dim must be <= 8192");
   if (1LL * c->batch * L > (1LL << 31) - 1) return fail(SA_ERR_UNSUPPORTED, "batch * chunk too big");
@@ -80,6 +91,8 @@ Derived derive(const sa_config& c) {
   d.W = c.window_chunks;
   d.R = d.W - 1;
   d.L = d.F * d.th * d.tw;
+  d.RF = c.ref_frames;
+  d.Lref = d.RF * d.th * d.tw;
   const int d_sp = 2 * (d.D / 6);
   d.dt2 = (d.D - 2 * d_sp) / 2;
   d.dh2 = d_sp / 2;
@@ -87,12 +100,13 @@ Derived derive(const sa_config& c) {
   d.scale = c.softmax_scale > 0.f ? c.softmax_scale : 1.f / std::sqrt(static_cast<float>(d.D));
   d.theta = c.rope_theta > 0.f ? c.rope_theta : 10000.f;
   d.chunk_elems = static_cast<size_t>(d.B) * d.H * d.L * d.D;
+  d.ref_elems = static_cast<size_t>(d.B) * d.H * d.Lref * d.D;
   const size_t slot_bytes = 2 * d.chunk_elems * sizeof(__nv_bfloat16);
   size_t off = 0;
   d.off_status = off;
   off += 1024;
   d.off_rope_t = off;
-  off += align_up(static_cast<size_t>(d.S + d.W) * d.F * d.dt2 * sizeof(float2), 1024);
+  off += align_up(static_cast<size_t>(d.RF + (d.S + d.W) * d.F) * d.dt2 * sizeof(float2), 1024);
   d.off_rope_h = off;
   off += align_up(static_cast<size_t>(d.th) * d.dh2 * sizeof(float2), 1024);
   d.off_rope_w = off;
@@ -103,6 +117,8 @@ Derived derive(const sa_config& c) {
   }
   d.off_kcur = off;
   off += align_up(d.chunk_elems * sizeof(__nv_bfloat16), 1024);
+  d.off_ref = off;
+  off += align_up(2 * d.ref_elems * sizeof(__nv_bfloat16), 1024);
   // split-tail scratch: partial rows, their lse, per-row merge counters
   const size_t split_rows = static_cast<size_t>(sa::kMaxSplitSlots) * 2 * 2 * 128;
   d.off_split_o = off;
@@ -161,23 +177,24 @@ bool encode_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* 
   return r == CUDA_SUCCESS;
 }
 
-// [planes][L][D] with planes contiguous L x D matrices.
-bool encode_planes(CUtensorMap* map, const void* base, const Derived& d, long long planes) {
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d.D), static_cast<cuuint64_t>(d.L),
+// [planes][rows][D] with planes contiguous rows x D matrices.
+bool encode_planes(CUtensorMap* map, const void* base, const Derived& d, int rows,
+                   long long planes) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d.D), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(planes)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d.D) * 2,
-                           static_cast<cuuint64_t>(d.L) * d.D * 2};
+                           static_cast<cuuint64_t>(rows) * d.D * 2};
   cuuint32_t box[3] = {64, 128, 1};
   return encode_map(map, base, 3, dims, strides, box);
 }
 
-// The caller's [B, L, H, D] tensor as (D, H, L, B).
-bool encode_blhd(CUtensorMap* map, const void* base, const Derived& d) {
+// The caller's [B, L, H, D] tensor (L = rows) as (D, H, L, B).
+bool encode_blhd(CUtensorMap* map, const void* base, const Derived& d, int rows) {
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(d.D), static_cast<cuuint64_t>(d.H),
-                        static_cast<cuuint64_t>(d.L), static_cast<cuuint64_t>(d.B)};
+                        static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(d.B)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(d.D) * 2,
                            static_cast<cuuint64_t>(d.H) * d.D * 2,
-                           static_cast<cuuint64_t>(d.L) * d.H * d.D * 2};
+                           static_cast<cuuint64_t>(rows) * d.H * d.D * 2};
   cuuint32_t box[4] = {64, 1, 128, 1};
   return encode_map(map, base, 4, dims, strides, box);
 }
@@ -186,8 +203,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // Persistent grid: one CTA per SM at most; with the split tail allowed, a problem
 // of fewer work tiles than SMs gets two CTAs per tile (key-range halves).
-unsigned attend_grid(const Derived& d, int sm_count, bool split_ok) {
-  const int n_qt = (d.L + 127) / 128;
+unsigned attend_grid(const Derived& d, int rows, int sm_count, bool split_ok) {
+  const int n_qt = (rows + 127) / 128;
   const long long n_work = 1LL * d.B * d.H * ((n_qt + 1) / 2);
   long long g = n_work < sm_count ? n_work : sm_count;
   if (split_ok && n_work < sm_count) g = 2 * n_work < sm_count ? 2 * n_work : sm_count;
@@ -195,21 +212,29 @@ unsigned attend_grid(const Derived& d, int sm_count, bool split_ok) {
 }
 
 // The attention kernel instantiations: head dim 128 / 64, dense / block-sparse.
+// Tensor maps of one launch: cache tier, key scratch, current V, reference.
+struct AttendMaps {
+  const CUtensorMap* cache;
+  const CUtensorMap* kcur;
+  const CUtensorMap* vcur;
+  const CUtensorMap* ref;
+};
+
 template <int D, bool kSparse>
-void launch_attend_tc_t(unsigned grid, cudaStream_t s, const CUtensorMap& a, const CUtensorMap& b,
-                        const CUtensorMap& c, const AttendParams& ap) {
-  sa::attend_tc_kernel<D, kSparse>
-      <<<grid, sa::TcShape<D>::kThreads, sa::TcShape<D>::kSmemBytes, s>>>(a, b, c, ap);
+void launch_attend_tc_t(unsigned grid, cudaStream_t s, const AttendMaps& m,
+                        const AttendParams& ap) {
+  sa::attend_tc_kernel<D, kSparse><<<grid, sa::TcShape<D>::kThreads, sa::TcShape<D>::kSmemBytes,
+                                     s>>>(*m.cache, *m.kcur, *m.vcur, *m.ref, ap);
 }
 
-void launch_attend_tc(int D, bool sparse, unsigned grid, cudaStream_t s, const CUtensorMap& a,
-                      const CUtensorMap& b, const CUtensorMap& c, const AttendParams& ap) {
+void launch_attend_tc(int D, bool sparse, unsigned grid, cudaStream_t s, const AttendMaps& m,
+                      const AttendParams& ap) {
   if (D == 128)
-    sparse ? launch_attend_tc_t<128, true>(grid, s, a, b, c, ap)
-           : launch_attend_tc_t<128, false>(grid, s, a, b, c, ap);
+    sparse ? launch_attend_tc_t<128, true>(grid, s, m, ap)
+           : launch_attend_tc_t<128, false>(grid, s, m, ap);
   else
-    sparse ? launch_attend_tc_t<64, true>(grid, s, a, b, c, ap)
-           : launch_attend_tc_t<64, false>(grid, s, a, b, c, ap);
+    sparse ? launch_attend_tc_t<64, true>(grid, s, m, ap)
+           : launch_attend_tc_t<64, false>(grid, s, m, ap);
 }
 
 // Every instantiation: the register count the setmaxnreg split assumes, and the
@@ -239,10 +264,14 @@ struct sa_handle {
   int sm_count;
   uint8_t* buf;
   int count[2];
-  int staged_chunk;  // chunk whose keys sit in the scratch (-1: none)
+  int frames[2][SA_MAX_ATTENDED];  // frames of the chunk each slot holds, per tier
+  int staged_chunk;                // chunk whose keys sit in the scratch (-1: none)
+  int staged_frames;               // its frames
   bool has_cache;
+  bool has_ref;  // a reference image is set
   CUtensorMap tm_tier[2];
   CUtensorMap tm_kcur;
+  CUtensorMap tm_ref;
   std::string err;
 
   int fail(int code, const std::string& msg) {
@@ -252,6 +281,7 @@ struct sa_handle {
   unsigned* status() { return reinterpret_cast<unsigned*>(buf + d.off_status); }
   __nv_bfloat16* tier_base(int t) { return reinterpret_cast<__nv_bfloat16*>(buf + d.off_tier[t]); }
   __nv_bfloat16* kcur() { return reinterpret_cast<__nv_bfloat16*>(buf + d.off_kcur); }
+  __nv_bfloat16* ref() { return reinterpret_cast<__nv_bfloat16*>(buf + d.off_ref); }
   RopeTables rope() {
     RopeTables rt;
     rt.t = reinterpret_cast<const float2*>(buf + d.off_rope_t);
@@ -277,8 +307,9 @@ int check_device(sa_handle* h) {
   return SA_OK;
 }
 
+// Rotate K (and copy V, if given) of `rows` tokens into [B, H, L_out, D] planes.
 int launch_rope_transpose(sa_handle* h, const void* K, const void* V, __nv_bfloat16* k_out,
-                          __nv_bfloat16* v_out, cudaStream_t s) {
+                          __nv_bfloat16* v_out, int rows, int L_out, cudaStream_t s) {
   const Derived& d = h->d;
   AppendParams ap;
   ap.k_in = static_cast<const __nv_bfloat16*>(K);
@@ -286,12 +317,13 @@ int launch_rope_transpose(sa_handle* h, const void* K, const void* V, __nv_bfloa
   ap.k_out = k_out;
   ap.v_out = v_out;
   ap.B = d.B;
-  ap.L = d.L;
+  ap.L = rows;
   ap.H = d.H;
   ap.D = d.D;
+  ap.L_out = L_out;
   ap.rope = h->rope();
   const int threads = static_cast<int>(align_up(static_cast<size_t>(d.H) * d.D / 8, 32));
-  dim3 grid(static_cast<unsigned>(d.B) * d.L, V != nullptr ? 2 : 1);
+  dim3 grid(static_cast<unsigned>(d.B) * rows, V != nullptr ? 2 : 1);
   sa::rope_transpose_kernel<<<grid, threads, 0, s>>>(ap);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
@@ -307,8 +339,101 @@ int check_handle(sa_handle* h) {
   return SA_OK;
 }
 
-int stage_keys(sa_handle* h, const void* Kc, sa_stream stream) {
+int check_frames(sa_handle* h, int n_frames) {
+  if (n_frames < 1 || n_frames > h->d.F)
+    return h->fail(SA_ERR_INVALID_ARG, "n_frames must be in 1..frames_per_chunk");
+  return SA_OK;
+}
+
+// The attention plan of the generating chunk c (n_frames frames) on `tier`:
+// attended chunk ids in ascending order, each with its cache slot (-1: the chunk
+// itself), frames and relocated temporal base = ref_frames + the frames of the
+// attended chunks before it.
+struct Plan {
+  int n;
+  int ids[SA_MAX_ATTENDED], slot[SA_MAX_ATTENDED], frames[SA_MAX_ATTENDED],
+      base[SA_MAX_ATTENDED];
+};
+
+Plan make_plan(const sa_handle* h, int tier, int n_frames) {
+  const Derived& d = h->d;
+  const int c = h->count[0];
+  Plan pl;
+  pl.n = plan_ids(d, c, pl.ids);
+  int pos = d.RF;
+  for (int g = 0; g < pl.n; ++g) {
+    const int id = pl.ids[g];
+    pl.slot[g] = id == c ? -1 : slot_of(d, id);
+    pl.frames[g] = id == c ? n_frames : h->frames[tier][pl.slot[g]];
+    pl.base[g] = pos;
+    pos += pl.frames[g];
+  }
+  return pl;
+}
+
+// Key groups of the attention kernels: the reference image (if set), then the
+// plan's chunks. t_delta = base(current) - base(group) >= 0.
+void fill_groups(const sa_handle* h, int tier, int n_frames, AttendParams* ap) {
+  const Derived& d = h->d;
+  const Plan pl = make_plan(h, tier, n_frames);
+  const int base_c = pl.base[pl.n - 1];
+  int n = 0;
+  if (h->has_ref) {
+    AttendGroup& grp = ap->groups[n++];
+    grp.src = 2;
+    grp.slot = 0;
+    grp.t_delta = base_c;
+    grp.len = d.Lref;
+  }
+  for (int g = 0; g < pl.n; ++g) {
+    AttendGroup& grp = ap->groups[n++];
+    grp.src = pl.slot[g] < 0 ? 1 : 0;
+    grp.slot = pl.slot[g] < 0 ? 0 : pl.slot[g];
+    grp.t_delta = base_c - pl.base[g];
+    grp.len = pl.frames[g] * d.th * d.tw;
+  }
+  ap->n_groups = n;
+}
+
+// Everything of AttendParams but the key source of the current chunk.
+void fill_common(sa_handle* h, int tier, int n_frames, const void* Q, const void* Vc, void* O,
+                 float* lse, AttendParams* ap) {
+  const Derived& d = h->d;
+  std::memset(ap, 0, sizeof(*ap));
+  ap->q = static_cast<const __nv_bfloat16*>(Q);
+  ap->o = static_cast<__nv_bfloat16*>(O);
+  ap->lse = lse;
+  ap->cache = h->tier_base(tier);
+  ap->v_cur = static_cast<const __nv_bfloat16*>(Vc);
+  ap->ref = h->has_ref ? h->ref() : nullptr;
+  ap->B = d.B;
+  ap->L = n_frames * d.th * d.tw;
+  ap->H = d.H;
+  ap->D = d.D;
+  ap->L_plane = d.L;
+  ap->L_ref = d.Lref;
+  fill_groups(h, tier, n_frames, ap);
+  ap->scale_log2 = d.scale * 1.4426950408889634f;
+  ap->rope = h->rope();
+  ap->status = h->status();
+}
+
+int check_attend_ptrs(sa_handle* h, const void* Q, const void* Vc, const void* O,
+                      const float* lse) {
+  if (Q == nullptr || Vc == nullptr || O == nullptr)
+    return h->fail(SA_ERR_INVALID_ARG, "Q, Vc and O must be non-NULL");
+  if (!aligned16(Q) || !aligned16(Vc) || !aligned16(O))
+    return h->fail(SA_ERR_INVALID_ARG, "Q, Vc and O must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+    return h->fail(SA_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+  if (O == Q || O == Vc) return h->fail(SA_ERR_INVALID_ARG, "O must not alias an input");
+  return SA_OK;
+}
+
+int stage_keys(sa_handle* h, const void* Kc, int n_frames, sa_stream stream) {
   int rc = check_handle(h);
+  if (rc != SA_OK) return rc;
+  rc = check_frames(h, n_frames);
   if (rc != SA_OK) return rc;
   if (Kc == nullptr || !aligned16(Kc))
     return h->fail(SA_ERR_INVALID_ARG, "Kc must be a non-NULL 16-byte aligned pointer");
@@ -316,10 +441,11 @@ int stage_keys(sa_handle* h, const void* Kc, sa_stream stream) {
     return h->fail(SA_ERR_STATE, "both tiers must hold the same chunks before attending");
   rc = check_device(h);
   if (rc != SA_OK) return rc;
-  rc = launch_rope_transpose(h, Kc, nullptr, h->kcur(), nullptr,
-                             reinterpret_cast<cudaStream_t>(stream));
+  rc = launch_rope_transpose(h, Kc, nullptr, h->kcur(), nullptr, n_frames * h->d.th * h->d.tw,
+                             h->d.L, reinterpret_cast<cudaStream_t>(stream));
   if (rc != SA_OK) return rc;
   h->staged_chunk = h->count[0];
+  h->staged_frames = n_frames;
   return SA_OK;
 }
 
@@ -328,49 +454,23 @@ int attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final
                   const uint8_t* block_mask = nullptr) {
   int rc = check_handle(h);
   if (rc != SA_OK) return rc;
-  if (Q == nullptr || Vc == nullptr || O == nullptr)
-    return h->fail(SA_ERR_INVALID_ARG, "Q, Vc and O must be non-NULL");
-  if (!aligned16(Q) || !aligned16(Vc) || !aligned16(O))
-    return h->fail(SA_ERR_INVALID_ARG, "Q, Vc and O must be 16-byte aligned");
-  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
-    return h->fail(SA_ERR_INVALID_ARG, "lse must be 4-byte aligned");
-  if (O == Q || O == Vc) return h->fail(SA_ERR_INVALID_ARG, "O must not alias an input");
+  rc = check_attend_ptrs(h, Q, Vc, O, lse);
+  if (rc != SA_OK) return rc;
   if (h->count[0] != h->count[1])
     return h->fail(SA_ERR_STATE, "both tiers must hold the same chunks before attending");
   if (h->staged_chunk != h->count[0])
     return h->fail(SA_ERR_STATE, "no keys staged for the current chunk (call sa_stage_keys)");
+  if (block_mask != nullptr && h->has_ref)
+    return h->fail(SA_ERR_UNSUPPORTED, "block-sparse attention takes no reference image");
   rc = check_device(h);
   if (rc != SA_OK) return rc;
   const Derived& d = h->d;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int tier = step_is_final ? SA_TIER_CLEAN : SA_TIER_NOISY;
-  const int c = h->count[0];
 
   AttendParams ap;
-  std::memset(&ap, 0, sizeof(ap));
-  ap.q = static_cast<const __nv_bfloat16*>(Q);
-  ap.o = static_cast<__nv_bfloat16*>(O);
-  ap.lse = lse;
-  ap.cache = h->tier_base(tier);
+  fill_common(h, tier, h->staged_frames, Q, Vc, O, lse, &ap);
   ap.k_cur = h->kcur();
-  ap.v_cur = static_cast<const __nv_bfloat16*>(Vc);
-  ap.B = d.B;
-  ap.L = d.L;
-  ap.H = d.H;
-  ap.D = d.D;
-  int ids[SA_MAX_ATTENDED];
-  const int n = plan_ids(d, c, ids);
-  ap.n_groups = n;
-  for (int g = 0; g < n; ++g) {
-    AttendGroup& grp = ap.groups[g];
-    grp.src = ids[g] == c ? 1 : 0;
-    grp.slot = ids[g] == c ? 0 : slot_of(d, ids[g]);
-    grp.t_delta = (n - 1 - g) * d.F;
-    grp.len = d.L;
-  }
-  ap.scale_log2 = d.scale * 1.4426950408889634f;
-  ap.rope = h->rope();
-  ap.status = h->status();
   ap.debug_stall_producer = debug_stall ? 1 : 0;
   ap.block_mask = block_mask;
   ap.split_o = reinterpret_cast<float*>(h->buf + d.off_split_o);
@@ -379,7 +479,7 @@ int attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final
   ap.split_ok = h->sm_count <= 2 * sa::kMaxSplitSlots ? 1 : 0;
 
   if (simt) {
-    const long long rows = 1LL * d.B * d.H * d.L;
+    const long long rows = 1LL * d.B * d.H * ap.L;
     const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
     if (d.D == 128)
       sa::attend_simt_kernel<128><<<grid, 256, 0, s>>>(ap);
@@ -387,10 +487,11 @@ int attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final
       sa::attend_simt_kernel<64><<<grid, 256, 0, s>>>(ap);
   } else {
     CUtensorMap tm_v;
-    if (!encode_blhd(&tm_v, Vc, d)) return h->fail(SA_ERR_CUDA, "TMA descriptor for Vc failed");
-    const CUtensorMap& tm_cache = h->has_cache ? h->tm_tier[tier] : h->tm_kcur;
-    launch_attend_tc(d.D, block_mask != nullptr, attend_grid(d, h->sm_count, ap.split_ok != 0), s,
-                     tm_cache, h->tm_kcur, tm_v, ap);
+    if (!encode_blhd(&tm_v, Vc, d, ap.L)) return h->fail(SA_ERR_CUDA, "TMA descriptor for Vc failed");
+    AttendMaps maps{h->has_cache ? &h->tm_tier[tier] : &h->tm_kcur, &h->tm_kcur, &tm_v,
+                    d.RF > 0 ? &h->tm_ref : &h->tm_kcur};
+    launch_attend_tc(d.D, block_mask != nullptr,
+                     attend_grid(d, ap.L, h->sm_count, ap.split_ok != 0), s, maps, ap);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
@@ -398,21 +499,21 @@ int attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final
   return SA_OK;
 }
 
-int attend_common(sa_handle* h, const void* Q, const void* Kc, const void* Vc, int step_is_final,
-                  void* O, float* lse, sa_stream stream, bool simt) {
+int attend_common(sa_handle* h, const void* Q, const void* Kc, const void* Vc, int n_frames,
+                  int step_is_final, void* O, float* lse, sa_stream stream, bool simt,
+                  const uint8_t* block_mask = nullptr) {
   int rc = check_handle(h);
   if (rc != SA_OK) return rc;
-  if (Q == nullptr || Kc == nullptr || Vc == nullptr || O == nullptr)
-    return h->fail(SA_ERR_INVALID_ARG, "Q, Kc, Vc and O must be non-NULL");
+  if (Kc == nullptr) return h->fail(SA_ERR_INVALID_ARG, "Kc must be non-NULL");
   if (O == Kc) return h->fail(SA_ERR_INVALID_ARG, "O must not alias an input");
   // Validate the attention half before launching the staging half.
-  if (!aligned16(Q) || !aligned16(Vc) || !aligned16(O) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 || O == Q || O == Vc)
-    return h->fail(SA_ERR_INVALID_ARG, "Q, Vc, O must be 16-byte aligned, lse 4-byte aligned, "
-                                       "O must not alias an input");
-  rc = stage_keys(h, Kc, stream);
+  rc = check_attend_ptrs(h, Q, Vc, O, lse);
   if (rc != SA_OK) return rc;
-  return attend_staged(h, Q, Vc, step_is_final, O, lse, stream, simt);
+  if (block_mask != nullptr && h->has_ref)
+    return h->fail(SA_ERR_UNSUPPORTED, "block-sparse attention takes no reference image");
+  rc = stage_keys(h, Kc, n_frames, stream);
+  if (rc != SA_OK) return rc;
+  return attend_staged(h, Q, Vc, step_is_final, O, lse, stream, simt, false, block_mask);
 }
 
 // ---------------------------------------------------------------- sa_attend_noalloc
@@ -446,12 +547,10 @@ int attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc, 
                    void* O, float* lse, sa_stream stream) {
   int rc = check_handle(h);
   if (rc != SA_OK) return rc;
-  if (Q == nullptr || Kc == nullptr || Vc == nullptr || O == nullptr)
-    return h->fail(SA_ERR_INVALID_ARG, "Q, Kc, Vc and O must be non-NULL");
-  if (!aligned16(Q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(O) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 || O == Q || O == Kc || O == Vc)
-    return h->fail(SA_ERR_INVALID_ARG, "Q, Kc, Vc, O must be 16-byte aligned, lse 4-byte "
-                                       "aligned, O must not alias an input");
+  if (Kc == nullptr || !aligned16(Kc) || O == Kc)
+    return h->fail(SA_ERR_INVALID_ARG, "Kc must be non-NULL, 16-byte aligned, not aliased by O");
+  rc = check_attend_ptrs(h, Q, Vc, O, lse);
+  if (rc != SA_OK) return rc;
   if (h->count[0] != h->count[1])
     return h->fail(SA_ERR_STATE, "both tiers must hold the same chunks before attending");
   const Derived& d = h->d;
@@ -466,49 +565,69 @@ int attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc, 
   __nv_bfloat16* keys = static_cast<__nv_bfloat16*>(scratch);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int tier = step_is_final ? SA_TIER_CLEAN : SA_TIER_NOISY;
-  const int c = h->count[0];
 
   CUtensorMap tm_keys, tm_v;
-  if (!encode_planes(&tm_keys, keys, d, 1LL * d.B * d.H) || !encode_blhd(&tm_v, Vc, d))
+  if (!encode_planes(&tm_keys, keys, d, d.L, 1LL * d.B * d.H) || !encode_blhd(&tm_v, Vc, d, d.L))
     return h->fail(SA_ERR_CUDA, "TMA descriptors for sa_attend_noalloc failed");
 
   AttendParams ap;
-  std::memset(&ap, 0, sizeof(ap));
-  ap.q = static_cast<const __nv_bfloat16*>(Q);
-  ap.o = static_cast<__nv_bfloat16*>(O);
-  ap.lse = lse;
-  ap.cache = h->tier_base(tier);
+  fill_common(h, tier, d.F, Q, Vc, O, lse, &ap);
   ap.k_cur = keys;
-  ap.v_cur = static_cast<const __nv_bfloat16*>(Vc);
-  ap.B = d.B;
-  ap.L = d.L;
-  ap.H = d.H;
-  ap.D = d.D;
-  int ids[SA_MAX_ATTENDED];
-  const int n = plan_ids(d, c, ids);
-  ap.n_groups = n;
-  for (int g = 0; g < n; ++g) {
-    AttendGroup& grp = ap.groups[g];
-    grp.src = ids[g] == c ? 1 : 0;
-    grp.slot = ids[g] == c ? 0 : slot_of(d, ids[g]);
-    grp.t_delta = (n - 1 - g) * d.F;
-    grp.len = d.L;
-  }
-  ap.scale_log2 = d.scale * 1.4426950408889634f;
-  ap.rope = h->rope();
-  ap.status = h->status();
+  ap.split_ok = 0;  // no scratch but the fixed key array: no split tail
 
   // Every element of the scratch that the attention reads is written first by
-  // this launch, so nothing has to start at zero.
-  rc = launch_rope_transpose(h, Kc, nullptr, keys, nullptr, s);
+  // this launch, or lies past the chunk's keys and is masked.
+  rc = launch_rope_transpose(h, Kc, nullptr, keys, nullptr, d.L, d.L, s);
   if (rc != SA_OK) return rc;
-  const CUtensorMap& tm_cache = h->has_cache ? h->tm_tier[tier] : tm_keys;
-  ap.split_ok = 0;  // no scratch but the fixed key array: no split tail
-  launch_attend_tc(d.D, false, attend_grid(d, h->sm_count, false), s, tm_cache, tm_keys, tm_v,
-                   ap);
+  AttendMaps maps{h->has_cache ? &h->tm_tier[tier] : &tm_keys, &tm_keys, &tm_v,
+                  d.RF > 0 ? &h->tm_ref : &tm_keys};
+  launch_attend_tc(d.D, false, attend_grid(d, d.L, h->sm_count, false), s, maps, ap);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
     return h->fail(SA_ERR_CUDA, std::string("attend launch: ") + cudaGetErrorString(e));
+  return SA_OK;
+}
+
+int append_chunk(sa_handle* h, int tier, const void* K, const void* V, int n_frames,
+                 sa_stream stream) {
+  int rc = check_handle(h);
+  if (rc != SA_OK) return rc;
+  if (tier != SA_TIER_NOISY && tier != SA_TIER_CLEAN)
+    return h->fail(SA_ERR_INVALID_ARG, "tier must be SA_TIER_NOISY or SA_TIER_CLEAN");
+  rc = check_frames(h, n_frames);
+  if (rc != SA_OK) return rc;
+  if (K == nullptr || V == nullptr) return h->fail(SA_ERR_INVALID_ARG, "K and V must be non-NULL");
+  if (!aligned16(K) || !aligned16(V))
+    return h->fail(SA_ERR_INVALID_ARG, "K and V must be 16-byte aligned");
+  if (h->count[tier] > h->count[1 - tier])
+    return h->fail(SA_ERR_STATE, "this tier is already one chunk ahead of the other");
+  rc = check_device(h);
+  if (rc != SA_OK) return rc;
+  const Derived& d = h->d;
+  const int id = h->count[tier];
+  const int slot = slot_of(d, id);
+  if (slot >= 0) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    __nv_bfloat16* base = h->tier_base(tier) + static_cast<size_t>(slot) * 2 * d.chunk_elems;
+    const int rows = n_frames * d.th * d.tw;
+    rc = launch_rope_transpose(h, K, V, base, base + d.chunk_elems, rows, d.L, s);
+    if (rc != SA_OK) return rc;
+    // A short chunk's last key tile reads V rows past its end: P is 0 there, so
+    // they only need to be finite. Zero them up to the tile boundary (the slot
+    // may never have been written).
+    const int hi = std::min(d.L, (rows + 127) / 128 * 128);
+    if (hi > rows) {
+      const size_t row_bytes = static_cast<size_t>(d.D) * sizeof(__nv_bfloat16);
+      if (cudaMemset2DAsync(base + d.chunk_elems + static_cast<size_t>(rows) * d.D,
+                            static_cast<size_t>(d.L) * row_bytes, 0,
+                            static_cast<size_t>(hi - rows) * row_bytes,
+                            static_cast<size_t>(d.B) * d.H, s) != cudaSuccess)
+        return h->fail(SA_ERR_CUDA, std::string("clearing a short chunk's tail: ") +
+                                        cudaGetErrorString(cudaGetLastError()));
+    }
+    h->frames[tier][slot] = n_frames;
+  }
+  h->count[tier] = id + 1;
   return SA_OK;
 }
 
@@ -576,10 +695,16 @@ SA_API int sa_create(const sa_config* cfg, void* dev_buf, size_t bytes, sa_handl
   h->sm_count = sms;
   h->buf = static_cast<uint8_t*>(dev_buf);
   h->count[0] = h->count[1] = 0;
+  for (int t = 0; t < 2; ++t)
+    for (int s = 0; s < SA_MAX_ATTENDED; ++s) h->frames[t][s] = d.F;
   h->staged_chunk = -1;
+  h->staged_frames = d.F;
+  h->has_ref = false;
 
   // RoPE tables: angle pos * theta^(-2i/d) in double, cos/sin cast to float.
-  std::vector<float2> t(static_cast<size_t>(d.S + d.W) * d.F * d.dt2);
+  // Temporal positions run over the reference frames and S + W chunks.
+  const int n_tpos = d.RF + (d.S + d.W) * d.F;
+  std::vector<float2> t(static_cast<size_t>(n_tpos) * d.dt2);
   std::vector<float2> th(static_cast<size_t>(d.th) * d.dh2), tw(static_cast<size_t>(d.tw) * d.dw2);
   auto fill = [&](std::vector<float2>& tab, int npos, int npair) {
     const double band = 2.0 * npair;
@@ -590,7 +715,7 @@ SA_API int sa_create(const sa_config* cfg, void* dev_buf, size_t bytes, sa_handl
             make_float2(static_cast<float>(std::cos(a)), static_cast<float>(std::sin(a)));
       }
   };
-  fill(t, (d.S + d.W) * d.F, d.dt2);
+  fill(t, n_tpos, d.dt2);
   fill(th, d.th, d.dh2);
   fill(tw, d.tw, d.dw2);
   bool ok = cudaMemset(h->buf + d.off_status, 0, 1024) == cudaSuccess &&
@@ -609,14 +734,20 @@ SA_API int sa_create(const sa_config* cfg, void* dev_buf, size_t bytes, sa_handl
   h->has_cache = d.S + d.R > 0;
   if (h->has_cache) {
     for (int tier = 0; tier < 2; ++tier)
-      if (!encode_planes(&h->tm_tier[tier], h->tier_base(tier), d, 2LL * (d.S + d.R) * d.B * d.H)) {
+      if (!encode_planes(&h->tm_tier[tier], h->tier_base(tier), d, d.L,
+                         2LL * (d.S + d.R) * d.B * d.H)) {
         g_error = "TMA descriptor for the cache failed";
         delete h;
         return SA_ERR_CUDA;
       }
   }
-  if (!encode_planes(&h->tm_kcur, h->kcur(), d, 1LL * d.B * d.H)) {
+  if (!encode_planes(&h->tm_kcur, h->kcur(), d, d.L, 1LL * d.B * d.H)) {
     g_error = "TMA descriptor for the key scratch failed";
+    delete h;
+    return SA_ERR_CUDA;
+  }
+  if (d.RF > 0 && !encode_planes(&h->tm_ref, h->ref(), d, d.Lref, 2LL * d.B * d.H)) {
+    g_error = "TMA descriptor for the reference image failed";
     delete h;
     return SA_ERR_CUDA;
   }
@@ -645,7 +776,10 @@ SA_API int sa_reset(sa_handle* h) {
   int rc = check_device(h);
   if (rc != SA_OK) return rc;
   h->count[0] = h->count[1] = 0;
+  for (int t = 0; t < 2; ++t)
+    for (int s = 0; s < SA_MAX_ATTENDED; ++s) h->frames[t][s] = h->d.F;
   h->staged_chunk = -1;
+  h->has_ref = false;
   if (cudaMemset(h->buf + h->d.off_status, 0, 1024) != cudaSuccess ||
       cudaMemset(h->buf + h->d.off_split_sem, 0, h->d.split_sem_bytes) != cudaSuccess ||
       cudaDeviceSynchronize() != cudaSuccess)
@@ -655,38 +789,54 @@ SA_API int sa_reset(sa_handle* h) {
 
 SA_API int sa_append_chunk(sa_handle* h, int tier, const void* K, const void* V,
                            sa_stream stream) {
-  if (h == nullptr) {
-    g_error = "handle is NULL";
-    return SA_ERR_INVALID_ARG;
-  }
-  if (tier != SA_TIER_NOISY && tier != SA_TIER_CLEAN)
-    return h->fail(SA_ERR_INVALID_ARG, "tier must be SA_TIER_NOISY or SA_TIER_CLEAN");
-  if (K == nullptr || V == nullptr) return h->fail(SA_ERR_INVALID_ARG, "K and V must be non-NULL");
-  if (!aligned16(K) || !aligned16(V))
-    return h->fail(SA_ERR_INVALID_ARG, "K and V must be 16-byte aligned");
-  if (h->count[tier] > h->count[1 - tier])
-    return h->fail(SA_ERR_STATE, "this tier is already one chunk ahead of the other");
-  int rc = check_device(h);
+  if (h == nullptr) return check_handle(h);
+  return append_chunk(h, tier, K, V, h->d.F, stream);
+}
+
+SA_API int sa_append_chunk_frames(sa_handle* h, int tier, const void* K, const void* V,
+                                  int n_frames, sa_stream stream) {
+  return append_chunk(h, tier, K, V, n_frames, stream);
+}
+
+SA_API int sa_set_reference(sa_handle* h, const void* K, const void* V, sa_stream stream) {
+  int rc = check_handle(h);
   if (rc != SA_OK) return rc;
-  const int id = h->count[tier];
-  const int slot = slot_of(h->d, id);
-  if (slot >= 0) {
-    __nv_bfloat16* base = h->tier_base(tier) + static_cast<size_t>(slot) * 2 * h->d.chunk_elems;
-    rc = launch_rope_transpose(h, K, V, base, base + h->d.chunk_elems,
-                               reinterpret_cast<cudaStream_t>(stream));
-    if (rc != SA_OK) return rc;
+  if (K == nullptr && V == nullptr) {
+    h->has_ref = false;
+    return SA_OK;
   }
-  h->count[tier] = id + 1;
+  if (h->d.RF == 0)
+    return h->fail(SA_ERR_STATE, "the config has ref_frames == 0: no room for a reference image");
+  if (K == nullptr || V == nullptr || !aligned16(K) || !aligned16(V))
+    return h->fail(SA_ERR_INVALID_ARG, "K and V must both be non-NULL and 16-byte aligned");
+  rc = check_device(h);
+  if (rc != SA_OK) return rc;
+  rc = launch_rope_transpose(h, K, V, h->ref(), h->ref() + h->d.ref_elems, h->d.Lref, h->d.Lref,
+                             reinterpret_cast<cudaStream_t>(stream));
+  if (rc != SA_OK) return rc;
+  h->has_ref = true;
   return SA_OK;
 }
 
 SA_API int sa_attend(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
                      int step_is_final, void* O, float* lse, sa_stream stream) {
-  return attend_common(h, Q, Kc, Vc, step_is_final, O, lse, stream, false);
+  if (h == nullptr) return check_handle(h);
+  return attend_common(h, Q, Kc, Vc, h->d.F, step_is_final, O, lse, stream, false);
+}
+
+SA_API int sa_attend_frames(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
+                            int n_frames, int step_is_final, void* O, float* lse,
+                            sa_stream stream) {
+  return attend_common(h, Q, Kc, Vc, n_frames, step_is_final, O, lse, stream, false);
 }
 
 SA_API int sa_stage_keys(sa_handle* h, const void* Kc, sa_stream stream) {
-  return stage_keys(h, Kc, stream);
+  if (h == nullptr) return check_handle(h);
+  return stage_keys(h, Kc, h->d.F, stream);
+}
+
+SA_API int sa_stage_keys_frames(sa_handle* h, const void* Kc, int n_frames, sa_stream stream) {
+  return stage_keys(h, Kc, n_frames, stream);
 }
 
 SA_API int sa_attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final,
@@ -696,7 +846,8 @@ SA_API int sa_attend_staged(sa_handle* h, const void* Q, const void* Vc, int ste
 
 SA_API int sa_debug_attend_simt(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
                                 int step_is_final, void* O, float* lse, sa_stream stream) {
-  return attend_common(h, Q, Kc, Vc, step_is_final, O, lse, stream, true);
+  if (h == nullptr) return check_handle(h);
+  return attend_common(h, Q, Kc, Vc, h->d.F, step_is_final, O, lse, stream, true);
 }
 
 SA_API int sa_attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
@@ -710,15 +861,7 @@ SA_API int sa_attend_sparse(sa_handle* h, const void* Q, const void* Kc, const v
   int rc = check_handle(h);
   if (rc != SA_OK) return rc;
   if (block_mask == nullptr) return h->fail(SA_ERR_INVALID_ARG, "block_mask must be non-NULL");
-  if (Q == nullptr || Kc == nullptr || Vc == nullptr || O == nullptr)
-    return h->fail(SA_ERR_INVALID_ARG, "Q, Kc, Vc and O must be non-NULL");
-  if (!aligned16(Q) || !aligned16(Vc) || !aligned16(O) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 || O == Q || O == Vc || O == Kc)
-    return h->fail(SA_ERR_INVALID_ARG, "Q, Vc, O must be 16-byte aligned, lse 4-byte aligned, "
-                                       "O must not alias an input");
-  rc = stage_keys(h, Kc, stream);
-  if (rc != SA_OK) return rc;
-  return attend_staged(h, Q, Vc, step_is_final, O, lse, stream, false, false, block_mask);
+  return attend_common(h, Q, Kc, Vc, h->d.F, step_is_final, O, lse, stream, false, block_mask);
 }
 
 SA_API int sa_block_grid(const sa_config* cfg, int32_t chunk, int32_t* n_q_tiles,
@@ -738,7 +881,8 @@ SA_API int sa_block_grid(const sa_config* cfg, int32_t chunk, int32_t* n_q_tiles
 
 SA_API int sa_debug_attend_stalled(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
                                    int step_is_final, void* O, sa_stream stream) {
-  int rc = stage_keys(h, Kc, stream);
+  if (h == nullptr) return check_handle(h);
+  int rc = stage_keys(h, Kc, h->d.F, stream);
   if (rc != SA_OK) return rc;
   return attend_staged(h, Q, Vc, step_is_final, O, nullptr, stream, false, true);
 }
@@ -796,9 +940,37 @@ SA_API int sa_plan(const sa_config* cfg, int32_t chunk, int32_t* ids, int32_t* s
   for (int g = 0; g < n; ++g) {
     if (ids) ids[g] = tmp[g];
     if (slots) slots[g] = tmp[g] == chunk ? -1 : slot_of(d, tmp[g]);
-    if (t_base) t_base[g] = g * d.F;
+    if (t_base) t_base[g] = d.RF + g * d.F;
   }
   return n;
+}
+
+SA_API int sa_stream_plan(const sa_handle* h, int step_is_final, int n_frames, int32_t* ids,
+                          int32_t* t_base, int32_t* lens, int cap) {
+  if (h == nullptr) {
+    g_error = "handle is NULL";
+    return -SA_ERR_INVALID_ARG;
+  }
+  sa_handle* hm = const_cast<sa_handle*>(h);  // for the error text only
+  if (n_frames < 1 || n_frames > h->d.F) {
+    hm->err = "n_frames must be in 1..frames_per_chunk";
+    return -SA_ERR_INVALID_ARG;
+  }
+  if (h->count[0] != h->count[1]) {
+    hm->err = "both tiers must hold the same chunks before attending";
+    return -SA_ERR_STATE;
+  }
+  const Plan pl = make_plan(h, step_is_final ? SA_TIER_CLEAN : SA_TIER_NOISY, n_frames);
+  if (cap < pl.n) {
+    hm->err = "cap too small";
+    return -SA_ERR_INVALID_ARG;
+  }
+  for (int g = 0; g < pl.n; ++g) {
+    if (ids) ids[g] = pl.ids[g];
+    if (t_base) t_base[g] = pl.base[g];
+    if (lens) lens[g] = pl.frames[g] * h->d.th * h->d.tw;
+  }
+  return pl.n;
 }
 
 SA_API int sa_slot_of(const sa_config* cfg, int32_t chunk) {

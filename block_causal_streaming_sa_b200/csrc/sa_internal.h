@@ -19,14 +19,15 @@ constexpr unsigned kDevErrTimeout = 1u;
 // D - 4*(D/6), 2*(D/6), 2*(D/6) dims, pair i of a band of size d turned by
 // pos * theta^(-2i/d)). Row = position, column = pair index in the band.
 struct RopeTables {
-  const float2* t;  // [(S + W) * F][dt2]
+  const float2* t;  // [ref_frames + (S + W) * F][dt2]
   const float2* h;  // [tok_h][dh2]
   const float2* w;  // [tok_w][dw2]
   int dt2, dh2, dw2;
   int tok_h, tok_w, frame_tokens;  // frame_tokens = tok_h * tok_w
 };
 
-// Rotate-and-transpose of one chunk: in [B, L, H, D] -> out [B, H, L, D].
+// Rotate-and-transpose of one chunk (or the reference image): in [B, L, H, D]
+// -> out [B, H, L_out, D] (planes of L_out >= L rows; rows L.. untouched).
 // K rows (bf16) are turned by their in-chunk (frame, row, column) position and
 // written as fp16; V rows (blockIdx.y == 1) are copied as bf16.
 struct AppendParams {
@@ -35,14 +36,17 @@ struct AppendParams {
   __nv_bfloat16* k_out;
   __nv_bfloat16* v_out;
   int B, L, H, D;
+  int L_out;  // rows per output plane
   RopeTables rope;
 };
 
-// One attended chunk, in ascending chunk-id order.
+// One attended key group: the reference image first (if set), then the
+// attended chunks in ascending chunk-id order.
 struct AttendGroup {
-  int src;      // 0: cache slot of the selected tier, 1: the chunk being generated
+  int src;      // 0: cache slot of the selected tier, 1: the chunk being generated,
+                // 2: the reference image
   int slot;     // cache slot (src == 0)
-  int t_delta;  // (rank(current) - rank(this chunk)) * F, >= 0
+  int t_delta;  // temporal base of the current chunk minus this group's, >= 0
   int len;      // number of keys
 };
 
@@ -50,11 +54,15 @@ struct AttendParams {
   const __nv_bfloat16* q;        // [B, L, H, D] unrotated
   __nv_bfloat16* o;              // [B, L, H, D]
   float* lse;                    // [B, H, L] or null
-  const __nv_bfloat16* cache;    // selected tier: [slot][K|V][B][H][L][D]; K planes hold
-                                 // fp16 keys rotated in-chunk, V planes bf16
-  const __nv_bfloat16* k_cur;    // current chunk K (fp16 bits), rotated in-chunk: [B][H][L][D]
+  const __nv_bfloat16* cache;    // selected tier: [slot][K|V][B][H][L_plane][D]; K planes
+                                 // hold fp16 keys rotated in-chunk, V planes bf16
+  const __nv_bfloat16* k_cur;    // current chunk K (fp16 bits), rotated in-chunk:
+                                 // [B][H][L_plane][D]
   const __nv_bfloat16* v_cur;    // current chunk V as passed: [B][L][H][D]
-  int B, L, H, D;
+  const __nv_bfloat16* ref;      // reference image [K|V][B][H][L_ref][D] (K fp16) or null
+  int B, L, H, D;                // L: query rows of the current chunk
+  int L_plane;                   // rows per cache / key-scratch plane (F * tok_h * tok_w)
+  int L_ref;                     // rows per reference plane
   int n_groups;
   AttendGroup groups[kMaxGroups];
   float scale_log2;  // softmax scale * log2(e)

@@ -73,10 +73,13 @@ typedef struct {
                                chunk being generated; W - 1 are cached */
   float softmax_scale;      /* <= 0 selects 1/sqrt(D) */
   float rope_theta;         /* <= 0 selects 10000 */
+  int32_t ref_frames;       /* frames of the reference image, 0..1023 (0: none).
+                               Every chunk's temporal positions start after them,
+                               whether or not a reference is set. */
 } sa_config;
 
 /* Upper bounds of this build (checked by sa_validate_config). */
-#define SA_MAX_ATTENDED 16 /* S + W */
+#define SA_MAX_ATTENDED 16 /* S + W, and S + W + 1 when ref_frames > 0 */
 #define SA_MAX_CHUNK_LEN (1 << 22)
 
 /* Validate a config; SA_OK or SA_ERR_INVALID_ARG / SA_ERR_UNSUPPORTED. Host only. */
@@ -84,8 +87,9 @@ SA_API int sa_validate_config(const sa_config* cfg);
 
 /* Bytes of device memory sa_create needs for cfg (0 if cfg is invalid):
  * a status word, fp32 RoPE tables, both cache tiers ((S + W - 1) slots of K and
- * V each, layout [slot][K|V][B][H][L][D], K fp16, V bf16) and one rotated-key chunk of scratch
- * for the chunk being generated. Host only. */
+ * V each, layout [slot][K|V][B][H][L][D], K fp16, V bf16), one rotated-key chunk of scratch
+ * for the chunk being generated and, when ref_frames > 0, the reference image
+ * ([K|V][B][H][ref_frames * tok_h * tok_w][D]). Host only. */
 SA_API size_t sa_required_bytes(const sa_config* cfg);
 
 /* Create a handle over a caller-owned device buffer of at least
@@ -98,9 +102,9 @@ SA_API int sa_create(const sa_config* cfg, void* dev_buf, size_t bytes, sa_handl
 /* Release the handle (host memory only; the caller frees dev_buf). NULL is OK. */
 SA_API int sa_destroy(sa_handle* h);
 
-/* Forget every cached chunk and clear the device status word (start a new
- * stream). Enqueues one small memset on the default stream of the device and
- * waits for it; not for use inside graph capture. */
+/* Forget every cached chunk and the reference image, and clear the device
+ * status word (start a new stream). Enqueues one small memset on the default
+ * stream of the device and waits for it; not for use inside graph capture. */
 SA_API int sa_reset(sa_handle* h);
 
 /* Append the next chunk's K/V ([B, L, H, D], unrotated) to one tier.
@@ -117,14 +121,38 @@ SA_API int sa_reset(sa_handle* h);
 SA_API int sa_append_chunk(sa_handle* h, int tier, const void* K, const void* V,
                            sa_stream stream);
 
+/* sa_append_chunk for a chunk of n_frames <= F frames (K, V: [B, n_frames *
+ * tok_h * tok_w, H, D]). "Vidu S2 vs PixVerse R2", section 选择五: a chunk's
+ * length follows the control signal up to a cap; here the cap is F and the
+ * chunk keeps a whole slot. Later chunks' temporal positions follow from the
+ * frames actually stored (see sa_attend). n_frames outside [1, F] is
+ * SA_ERR_INVALID_ARG. sa_append_chunk is this call with n_frames = F. */
+SA_API int sa_append_chunk_frames(sa_handle* h, int tier, const void* K, const void* V,
+                                  int n_frames, sa_stream stream);
+
+/* Set, replace or (K = V = NULL) clear the reference image: K, V [B, ref_frames
+ * * tok_h * tok_w, H, D] bf16, unrotated. "Vidu S2：实时可交互、可编辑、可立体的视频生成",
+ * section 2.2: every chunk also sees a shared reference image; "Vidu S2 vs
+ * PixVerse R2" (Vidu S2's side): one shared reference keeps the subject's
+ * identity. The reference sits at temporal positions 0 .. ref_frames - 1 (keys
+ * rotated once here by their (frame, row, column)), ahead of every chunk; it
+ * has a single copy read at every denoising step and is attended by every
+ * chunk until replaced, cleared or sa_reset. Requires ref_frames > 0 in the
+ * config (else SA_ERR_STATE). Asynchronous on `stream`: attention calls on
+ * other streams must be ordered after it by the caller. */
+SA_API int sa_set_reference(sa_handle* h, const void* K, const void* V, sa_stream stream);
+
 /* Attention of the chunk being generated (chunk id c = number of chunks in
  * both tiers) at one denoising step:
  *   O = softmax(rope(Q) rope(K)^T * scale) V
  * over the keys of every cached sink and window chunk of the selected tier
  * (clean if step_is_final != 0, else noisy) followed by the chunk's own Kc/Vc,
- * all bidirectional inside the chunk. Chunk j sits at temporal position
- * rank(j) * F + frame, rank = index of j among the attended chunks in
- * ascending id order, so positions stay below (S + W) * F.
+ * all bidirectional inside the chunk, preceded by the reference image when
+ * one is set (sa_set_reference). Frame f of attended chunk j sits at temporal
+ * position ref_frames + (frames of the attended chunks before j) + f; with
+ * every chunk of F frames that is ref_frames + rank(j) * F + f, rank = index of
+ * j among the attended chunks in ascending id order, so positions stay below
+ * ref_frames + (S + W) * F.
  * Q, Kc, Vc: [B, L, H, D] bf16 (unrotated), read only. Rotated Q and K enter
  * the score MMA as fp16, P and V the output MMA as bf16; accumulation is fp32.
  * O: [B, L, H, D] bf16, fully overwritten (must not alias the inputs).
@@ -136,6 +164,13 @@ SA_API int sa_append_chunk(sa_handle* h, int tier, const void* K, const void* V,
 SA_API int sa_attend(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
                      int step_is_final, void* O, float* lse, sa_stream stream);
 
+/* sa_attend for a generating chunk of n_frames <= F frames: Q, Kc, Vc, O are
+ * [B, Lc, H, D] and lse [B, H, Lc] with Lc = n_frames * tok_h * tok_w.
+ * sa_attend is this call with n_frames = F. */
+SA_API int sa_attend_frames(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
+                            int n_frames, int step_is_final, void* O, float* lse,
+                            sa_stream stream);
+
 /* Block-sparse attention ("Vidu S2 vs PixVerse R2：实时视频的两条技术路线", section
  * 选择四：速度从哪里来: PixVerse R2 learns block-sparse attention and skips more than
  * 90 % of the blocks). Same as sa_attend, but only the blocks flagged in
@@ -143,9 +178,12 @@ SA_API int sa_attend(sa_handle* h, const void* Q, const void* Kc, const void* Vc
  * x 128 keys of the attended key sequence (the attended chunks in ascending id
  * order, each cut into 128-key tiles from its first token, the last tile of a
  * chunk possibly short). block_mask: device uint8 [B][H][n_q_tiles][n_k_tiles]
- * (nonzero = attended), from sa_block_grid for the current chunk; read only.
- * Key tiles no query tile of a 256-row pair needs are neither loaded nor
- * multiplied. A row that sees no key gets O = 0 and lse = -inf. */
+ * (nonzero = attended); read only. n_k_tiles is the sum over the attended chunks
+ * of ceil(keys / 128): sa_block_grid gives it when every chunk has F frames,
+ * sa_stream_plan's lens in general. Key tiles no query tile of a 256-row pair
+ * needs are neither loaded nor multiplied. A row that sees no key gets O = 0
+ * and lse = -inf. The reference image is not part of the block grid: with a
+ * reference set this call returns SA_ERR_UNSUPPORTED. */
 SA_API int sa_attend_sparse(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
                             int step_is_final, const uint8_t* block_mask, void* O, float* lse,
                             sa_stream stream);
@@ -159,10 +197,13 @@ SA_API int sa_block_grid(const sa_config* cfg, int32_t chunk, int32_t* n_q_tiles
  * sa_stage_keys rotates the generating chunk's Kc ([B, L, H, D] bf16) by its
  * in-chunk positions into the handle's key scratch (one HBM-bound kernel).
  * sa_attend_staged then runs the attention kernel over the cache and the staged
- * keys, with Vc read in place. sa_attend_staged requires a preceding
+ * keys, with Vc read in place (Q, Vc, O, lse of the staged chunk's frames). sa_attend_staged requires a preceding
  * sa_stage_keys for the same chunk (else SA_ERR_STATE); the staged keys stay
  * valid until the next sa_stage_keys / sa_attend on this handle. */
 SA_API int sa_stage_keys(sa_handle* h, const void* Kc, sa_stream stream);
+/* sa_stage_keys for a generating chunk of n_frames <= F frames; the following
+ * sa_attend_staged then takes Q, Vc, O, lse of n_frames frames. */
+SA_API int sa_stage_keys_frames(sa_handle* h, const void* Kc, int n_frames, sa_stream stream);
 SA_API int sa_attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final,
                             void* O, float* lse, sa_stream stream);
 
@@ -217,13 +258,23 @@ SA_API int sa_chunk_count(const sa_handle* h, int tier);
  * min(n, S + W - 1) slots; returns the number of slots written. Host only. */
 SA_API int sa_debug_layout(const sa_handle* h, int tier, int32_t* slot_chunk_ids, int n);
 
-/* The attention plan of chunk `chunk` of a stream with config cfg, computed on
- * the host with no handle and no device: writes, for each attended chunk in
- * ascending id order, its id, its cache slot (-1 for the chunk itself) and its
- * relocated temporal base rank * F. Returns the count (<= S + W) or a negative
- * sa_status if cap is too small. */
+/* The attention plan of chunk `chunk` of a stream with config cfg whose chunks
+ * all have F frames, computed on the host with no handle and no device: writes,
+ * for each attended chunk in ascending id order, its id, its cache slot (-1 for
+ * the chunk itself) and its relocated temporal base ref_frames + rank * F.
+ * Returns the count (<= S + W) or a negative sa_status if cap is too small. */
 SA_API int sa_plan(const sa_config* cfg, int32_t chunk, int32_t* ids, int32_t* slots,
                    int32_t* t_base, int cap);
+
+/* The attention plan the handle would run now for a generating chunk of
+ * n_frames frames at the given step (host only, no device work): for each
+ * attended chunk in ascending id order its id, its relocated temporal base
+ * (ref_frames + the frames of the attended chunks before it, from the frames
+ * the selected tier actually stored) and its number of keys. The reference
+ * image is not listed (it always sits at 0). Returns the count or a negative
+ * sa_status (tiers out of step, bad n_frames, cap too small). */
+SA_API int sa_stream_plan(const sa_handle* h, int step_is_final, int n_frames, int32_t* ids,
+                          int32_t* t_base, int32_t* lens, int cap);
 
 /* Slot of chunk id `chunk` in a tier (-1 if it is never stored). Host only. */
 SA_API int sa_slot_of(const sa_config* cfg, int32_t chunk);

@@ -115,3 +115,48 @@ def test_block_grid_matches_oracle_tiling(name):
         assert nq == -(-w.chunk_len // 128)
         assert nk == len(key_tiles([w.chunk_len] * len(model.attended())))
         model.append()
+
+
+def test_reference_config_validation_and_bytes():
+    assert sa.sa_validate_config(_cfg(ref_frames=1)) == sa.SA_OK
+    assert sa.sa_validate_config(_cfg(ref_frames=-1)) == sa.SA_ERR_INVALID_ARG
+    assert sa.sa_validate_config(_cfg(ref_frames=1024)) == sa.SA_ERR_INVALID_ARG
+    # the reference takes one of the SA_MAX_ATTENDED key groups
+    assert sa.sa_validate_config(_cfg(sink_chunks=6, window_chunks=10)) == sa.SA_OK
+    assert sa.sa_validate_config(_cfg(sink_chunks=6, window_chunks=10, ref_frames=1)) \
+        == sa.SA_ERR_UNSUPPORTED
+    assert sa.sa_validate_config(_cfg(sink_chunks=5, window_chunks=10, ref_frames=2)) == sa.SA_OK
+    base = sa.sa_required_bytes(_cfg())
+    with_ref = sa.sa_required_bytes(_cfg(ref_frames=2))
+    # K and V planes of 2 frames x 64 tokens x 2 heads x 64 dims, bf16
+    assert with_ref - base >= 2 * (2 * 64) * 2 * 64 * 2
+
+
+@pytest.mark.parametrize("ref_frames", [1, 4])
+def test_plan_bases_shift_by_reference_frames(ref_frames):
+    """sa_plan's bases equal the oracle's positions for whole-chunk streams."""
+    import numpy as np
+
+    from oracle.stream import CLEAN, NOISY, OracleConfig, StreamOracle
+
+    cfg = _cfg(sink_chunks=1, window_chunks=3, ref_frames=ref_frames)
+    ocfg = OracleConfig(1, 1, 64, 3, 8, 8, 1, 3, ref_frames=ref_frames)
+    orc = StreamOracle(ocfg)
+    blank = np.zeros((1, 3 * 64, 1, 1))
+    for c in range(10):
+        ids, _, tbase = sa.sa_plan(cfg, c)
+        o_ids, o_base = orc.positions(True, 3)
+        assert ids == o_ids
+        assert tbase == [o_base[j] for j in ids]
+        for tier in (NOISY, CLEAN):
+            orc.append(tier, blank, blank)
+
+
+def test_null_handle_new_calls_fail_cleanly():
+    lib = sa.lib()
+    assert lib.sa_append_chunk_frames(None, 0, None, None, 1, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_set_reference(None, None, None, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_attend_frames(None, None, None, None, 1, 0, None, None, None) \
+        == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_stage_keys_frames(None, None, 1, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_stream_plan(None, 0, 1, None, None, None, 16) < 0
