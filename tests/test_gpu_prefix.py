@@ -65,8 +65,9 @@ class PrefixPair:
         lse = torch.empty((self.B, self.H, L), dtype=torch.float32, device="cuda")
         if noalloc:
             out = torch.empty_like(Q, device="cuda")
-            sa.sa_attend_noalloc(self.gpu.handle, Q.cuda().data_ptr(), Kc.cuda().data_ptr(),
-                                 Vc.cuda().data_ptr(), final, out.data_ptr(), lse.data_ptr(),
+            Qd, Kd, Vd = Q.cuda(), Kc.cuda(), Vc.cuda()  # held until the kernel has run
+            sa.sa_attend_noalloc(self.gpu.handle, Qd.data_ptr(), Kd.data_ptr(), Vd.data_ptr(),
+                                 final, out.data_ptr(), lse.data_ptr(),
                                  torch.cuda.current_stream().cuda_stream)
         else:
             out = self.gpu.attend(Q.cuda(), Kc.cuda(), Vc.cuda(), final, lse=lse)
