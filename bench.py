@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--sparsity", type=float, default=0.0,
                     help="block-sparse mode: share of 128x128 blocks skipped (seeded random mask)")
+    ap.add_argument("--editing", action="store_true",
+                    help="frame-aligned editing attention (source frames of the chunk as extra keys)")
     ap.add_argument("--ref-frames", type=int, default=0,
                     help="frames of a reference image every chunk also attends (0: none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -309,7 +311,7 @@ def run_ours(args, w):
     barrier, max_over_ranks = ranks.barrier, ranks.max
 
     stream = torch.cuda.Stream(device=dev)
-    names = ("Q", "Kc", "Vc", "Kn", "Vn", "Kcl", "Vcl")
+    names = ("Q", "Kc", "Vc", "Kn", "Vn", "Kcl", "Vcl") + (("Ks", "Vs") if args.editing else ())
     pool_host = [{n: w.tensor(n, 100 + c, layer=rank).pin_memory() for n in names}
                  for c in range(2)]
     pool = [{n: t.to(dev) for n, t in s.items()} for s in pool_host]
@@ -333,6 +335,9 @@ def run_ours(args, w):
             layer.set_reference(Kref, Vref)
         torch.cuda.synchronize(dev)
         flops += 4.0 * w.batch * w.heads * w.chunk_len * ref_len * w.head_dim
+    if args.editing:
+        # every query row also sees the tok_h * tok_w source tokens of its own frame
+        flops += 4.0 * w.batch * w.heads * w.chunk_len * (w.tok_h * w.tok_w) * w.head_dim
     steps_per_chunk = w.steps
     attends_per_chunk = steps_per_chunk * w.layers
     appends_per_chunk = 2 * w.layers
@@ -365,7 +370,15 @@ def run_ours(args, w):
             final = k == steps_per_chunk - 1
             for layer in layers:
                 h = layer.handle
-                if block_mask is not None:
+                if args.editing:
+                    # editing: the staging of Kc and Ks is inside the timed call
+                    if ev is not None:
+                        ev[0][a].record(stream)
+                    sa.sa_attend_aligned(h, s["Q"].data_ptr(), s["Kc"].data_ptr(),
+                                         s["Vc"].data_ptr(), s["Ks"].data_ptr(),
+                                         s["Vs"].data_ptr(), w.frames, final, out.data_ptr(), 0,
+                                         sp)
+                elif block_mask is not None:
                     # sparse: the staging kernel is inside the timed attention call
                     if ev is not None:
                         ev[0][a].record(stream)
@@ -485,11 +498,13 @@ def run_ours(args, w):
             "parallelism": f"replicas{world}" if world > 1 else "single",
             "block_sparsity": args.sparsity,
             "ref_frames": args.ref_frames, "ref_tokens": ref_len,
+            "frame_aligned_editing": args.editing,
         },
         "roofline": {
             "bound": "tensor",
-            "kernel": "attend_tc_kernel<128>" + (" (sparse, timed with its staging kernel)"
-                                                 if block_mask is not None else ""),
+            "kernel": "attend_tc_kernel<128>" + (
+                " (sparse, timed with its staging kernel)" if block_mask is not None else
+                " (frame-aligned, timed with its staging kernel)" if args.editing else ""),
             "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "peak_kind": f"bf16 sustained ({peak_src})", "frac_of_burst_peak": achieved / burst,
             "traffic": kernel_traffic("attend_tc.cuh", w.name),

@@ -10,7 +10,8 @@ from ._binding import (  # noqa: F401
     SA_OK, SA_ERR_INVALID_ARG, SA_ERR_STATE, SA_ERR_UNSUPPORTED, SA_ERR_CUDA, SA_ERR_TIMEOUT,
     SA_TIER_NOISY, SA_TIER_CLEAN, SaConfig, SaError, make_config, lib, header_symbols,
     sa_validate_config, sa_required_bytes, sa_create, sa_destroy, sa_reset, sa_append_chunk,
-    sa_append_chunk_frames, sa_set_reference, sa_attend, sa_attend_frames, sa_stage_keys,
+    sa_append_chunk_frames, sa_set_reference, sa_attend, sa_attend_frames, sa_attend_aligned,
+    sa_stage_keys,
     sa_stage_keys_frames, sa_attend_staged, sa_debug_attend_simt, sa_attend_noalloc, sa_debug_exp2,
     sa_debug_attend_stalled, sa_attend_sparse, sa_block_grid,
     sa_chunk_count, sa_debug_layout, sa_plan, sa_stream_plan, sa_slot_of,

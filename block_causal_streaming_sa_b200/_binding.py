@@ -65,6 +65,7 @@ _SIGNATURES = {
     "sa_set_reference": (_I, [_P, _P, _P, _P]),
     "sa_attend": (_I, [_P, _P, _P, _P, _I, _P, _P, _P]),
     "sa_attend_frames": (_I, [_P, _P, _P, _P, _I, _I, _P, _P, _P]),
+    "sa_attend_aligned": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
     "sa_stage_keys": (_I, [_P, _P, _P]),
     "sa_stage_keys_frames": (_I, [_P, _P, _I, _P]),
     "sa_attend_staged": (_I, [_P, _P, _P, _I, _P, _P, _P]),
@@ -165,6 +166,13 @@ def sa_set_reference(handle, K, V, stream=0):
 def sa_attend_frames(handle, Q, Kc, Vc, n_frames, step_is_final, O, lse=0, stream=0):
     _check(lib().sa_attend_frames(handle, _P(Q), _P(Kc), _P(Vc), int(n_frames),
                                   int(bool(step_is_final)), _P(O), _P(lse or None), _P(stream)),
+           handle)
+
+
+def sa_attend_aligned(handle, Q, Kc, Vc, Ks, Vs, n_frames, step_is_final, O, lse=0, stream=0):
+    """Frame-aligned editing attention: the usual keys plus the same-frame source tokens."""
+    _check(lib().sa_attend_aligned(handle, _P(Q), _P(Kc), _P(Vc), _P(Ks), _P(Vs), int(n_frames),
+                                   int(bool(step_is_final)), _P(O), _P(lse or None), _P(stream)),
            handle)
 
 

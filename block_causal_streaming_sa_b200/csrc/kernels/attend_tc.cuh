@@ -6,9 +6,12 @@
 // set: "Vidu S2：实时可交互、可编辑、可立体的视频生成", section 2.2), the cached sink and
 // window chunks of one TwinCache tier and the chunk's own keys, with the
 // temporal RoPE base of chunk j relocated to ref_frames + the frames of the
-// attended chunks before it (rank(j) * F when all have F frames). With
-// kSparse, only the 128 x 128 blocks a caller flags are attended (section
-// 选择四：速度从哪里来: block-sparse attention with most blocks skipped).
+// attended chunks before it (rank(j) * F when all have F frames). Variants
+// (template kMode): dense; sparse, where only the 128 x 128 blocks a caller flags
+// are attended (section 选择四：速度从哪里来: block-sparse attention with most blocks
+// skipped); aligned, frame-aligned editing ("Vidu S2：实时可交互、可编辑、可立体的视频生成",
+// section 2.6): the dense key set plus the source frames of the generating
+// chunk, each query row seeing only the source frame of its own moment.
 //
 // Design (B200):
 //  * persistent CTAs, one per SM; a work tile is two 128-row query tiles of one
@@ -221,14 +224,18 @@ __device__ __noinline__ void epilogue(const AttendParams& p, uint32_t tO, bool a
   *sem = 0;  // ready for the next launch
 }
 
-template <int D, bool kSparse>
+template <int D, int kMode>
 __global__ void __launch_bounds__(384, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tm_cache,
                      const __grid_constant__ CUtensorMap tm_kcur,
                      const __grid_constant__ CUtensorMap tm_vcur,
                      const __grid_constant__ CUtensorMap tm_ref,
+                     const __grid_constant__ CUtensorMap tm_vsrc,
                      const __grid_constant__ AttendParams p) {
   using T = TcShape<D>;
+  constexpr bool kSparse = kMode == kModeSparse;    // caller-flagged 128 x 128 blocks
+  constexpr bool kAligned = kMode == kModeAligned;  // last group: same-frame source keys
+  constexpr bool kSkip = kMode != kModeDense;       // some key tiles of a unit are skipped
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = ptx::smem_addr(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -311,24 +318,43 @@ __global__ void __launch_bounds__(384, 1)
   auto g_lo = [&](int half) { return half == 1 ? sched[3] : 0; };
   auto g_hi = [&](int half) { return half == 0 ? sched[3] : p.n_groups; };
 
-  // Block sparsity: key tile kt of a work tile is visited when either of its two
-  // query tiles has the block flagged. Flag rows at mask offsets mo (query tile
-  // 2 * pair) and mo1 (its partner, -1 when the pair has a single tile).
+  // Skipped key tiles. Block sparsity: key tile kt of a work tile is visited
+  // when either of its two query tiles has the block flagged; flag rows at mask
+  // offsets mo (query tile 2 * pair) and mo1 (its partner, -1 when the pair has a
+  // single tile). Frame-aligned: of the last group (the source frames), only the
+  // tiles [mo, mo1) holding the frames of the work tile's rows are visited; every
+  // other group is visited whole.
   auto mask_rows = [&](int w, int& mo, int& mo1) {
     mo = mo1 = -1;
-    if (!kSparse) return;
-    const int bh = w / n_pairs, pair = w - bh * n_pairs;
-    mo = (bh * n_qt + 2 * pair) * n_kt_total;
-    mo1 = 2 * pair + 1 < n_qt ? mo + n_kt_total : -1;
+    if constexpr (kSparse) {
+      const int bh = w / n_pairs, pair = w - bh * n_pairs;
+      mo = (bh * n_qt + 2 * pair) * n_kt_total;
+      mo1 = 2 * pair + 1 < n_qt ? mo + n_kt_total : -1;
+    } else if constexpr (kAligned) {
+      const int pair = w % n_pairs;
+      const int hw = p.rope.frame_tokens;
+      const int q0 = 2 * pair * T::BM, q1 = min(q0 + 2 * T::BM, p.L) - 1;
+      const int gs = p.n_groups - 1;
+      mo = gstart[gs] + (q0 / hw) * hw / T::BN;
+      mo1 = gstart[gs] + (min((q1 / hw + 1) * hw, groups[gs].len) + T::BN - 1) / T::BN;
+    }
   };
   auto flag = [&](int off, int kt) -> bool {
     return off >= 0 && __ldg(p.block_mask + off + kt) != 0;
   };
+  // First visited flat key tile in [from, hi), or a value >= hi if none.
   auto next_visited = [&](int mo, int mo1, int from, int hi) {
-    if (!kSparse) return from;
-    int kt = from;
-    while (kt < hi && !(flag(mo, kt) || flag(mo1, kt))) ++kt;
-    return kt;
+    if constexpr (kSparse) {
+      int kt = from;
+      while (kt < hi && !(flag(mo, kt) || flag(mo1, kt))) ++kt;
+      return kt;
+    } else if constexpr (kAligned) {
+      if (from < gstart[p.n_groups - 1]) return from;
+      const int u = from < mo ? mo : from;
+      return u < mo1 && u < hi ? u : hi;
+    } else {
+      return from;
+    }
   };
 
   if (warp < 4) {
@@ -340,6 +366,7 @@ __global__ void __launch_bounds__(384, 1)
       ptx::tma_prefetch_desc(&tm_kcur);
       ptx::tma_prefetch_desc(&tm_vcur);
       if (groups[0].src == 2) ptx::tma_prefetch_desc(&tm_ref);
+      if (kAligned) ptx::tma_prefetch_desc(&tm_vsrc);
       int stage = 0;
       uint32_t phase = 0, filled_mask = 0, filled_parity = 0;
       bool ok = true;
@@ -352,8 +379,12 @@ __global__ void __launch_bounds__(384, 1)
         mask_rows(w, mo, mo1);
         for (int g = g_lo(half); ok && g < g_hi(half); ++g) {
           const AttendGroup grp = groups[g];
-          const int nkt = (grp.len + T::BN - 1) / T::BN;
-          for (int t = 0; ok && t < nkt; ++t) {
+          int t0 = 0, t1 = (grp.len + T::BN - 1) / T::BN;
+          if (kAligned && g == p.n_groups - 1) {
+            t0 = mo - gstart[g];
+            t1 = mo1 - gstart[g];
+          }
+          for (int t = t0; ok && t < t1; ++t) {
             if (kSparse && !(flag(mo, gstart[g] + t) || flag(mo1, gstart[g] + t))) continue;
             for (int kv = 0; kv < 2; ++kv) {
               if (!ptx::mbar_wait(bar(T::EMPTY(stage)), phase ^ 1u, abort_flag, p.status)) {
@@ -370,6 +401,13 @@ __global__ void __launch_bounds__(384, 1)
                 } else if (grp.src == 2) {
                   ptx::tma_load_3d(dst + kb * T::kBox, &tm_ref, full, kb * 64, t * T::BN,
                                    (kv * p.B + b) * p.H + h);
+                } else if (grp.src == 3) {  // source frames: keys in scratch half 1
+                  if (kv == 0)
+                    ptx::tma_load_3d(dst + kb * T::kBox, &tm_kcur, full, kb * 64, t * T::BN,
+                                     (p.B + b) * p.H + h);
+                  else
+                    ptx::tma_load_4d(dst + kb * T::kBox, &tm_vsrc, full, kb * 64, h, t * T::BN,
+                                     b);
                 } else if (kv == 0) {
                   ptx::tma_load_3d(dst + kb * T::kBox, &tm_kcur, full, kb * 64, t * T::BN,
                                    b * p.H + h);
@@ -435,7 +473,7 @@ __global__ void __launch_bounds__(384, 1)
         int mo, mo1;
         mask_rows(w, mo, mo1);
         int u = next_visited(mo, mo1, lo, hi);
-        if (kSparse && u >= hi) {  // no block flagged: nothing to multiply
+        if (kSkip && u >= hi) {  // no block flagged: nothing to multiply
           for (int i = 0; i < 2 && ok; ++i)
             ok = ptx::mbar_wait(bar(T::QREADY(i)), rr & 1, abort_flag, p.status);
           continue;
@@ -514,11 +552,12 @@ __global__ void __launch_bounds__(384, 1)
       const size_t row_off = ((static_cast<size_t>(b) * p.L + qr) * p.H + h) * D;
       const int glo = g_lo(half), ghi = g_hi(half);
       int mo = -1, mo1 = -1, own = -1;
-      if (kSparse) {
+      if (kSkip) {
         mask_rows(w, mo, mo1);
         own = i == 0 ? mo : mo1;
       }
       // First chunk with a visited key tile (the query tile is rotated for it).
+      // Frame-aligned units visit every group, the last one partly.
       int g0 = glo;
       bool any_tile = true;
       if (kSparse) {
@@ -547,8 +586,12 @@ __global__ void __launch_bounds__(384, 1)
       int kt = 0;  // key tiles processed in this unit
       for (int g = glo; ok && any_tile && g < ghi; ++g) {
         const int len = groups[g].len;
-        const int nkt = (len + T::BN - 1) / T::BN;
-        for (int t = 0; t < nkt; ++t) {
+        int t0 = 0, t1 = (len + T::BN - 1) / T::BN;
+        if (kAligned && g == p.n_groups - 1) {
+          t0 = mo - gstart[g];
+          t1 = mo1 - gstart[g];
+        }
+        for (int t = t0; t < t1; ++t) {
           if (kSparse && next_visited(mo, mo1, gstart[g] + t, gstart[g] + t + 1) != gstart[g] + t)
             continue;
           if (!ptx::mbar_wait(bar(T::SFULL(i)), s_phase, abort_flag, p.status)) {
@@ -558,18 +601,25 @@ __global__ void __launch_bounds__(384, 1)
           s_phase ^= 1u;
           ptx::tc_fence_after();
           if (!kSparse || flag(own, gstart[g] + t)) {
-            // The whole score row (128 fp32) in one round trip; keys past the chunk end masked.
-            const int nvalid = min(T::BN, len - t * T::BN);
+            // The whole score row (128 fp32) in one round trip; keys past the chunk end
+            // masked, and in a source tile every key outside the row's own frame.
+            int c_lo = 0, c_hi = min(T::BN, len - t * T::BN);
+            if (kAligned && g == p.n_groups - 1) {
+              const int k0 = t * T::BN - f * p.rope.frame_tokens;  // tile start - frame start
+              c_lo = max(c_lo, -k0);
+              c_hi = min(c_hi, p.rope.frame_tokens - k0);
+            }
             uint32_t sr[4][32];
 #pragma unroll
             for (int j = 0; j < 4; ++j) ptx::tmem_ld32(tS + j * 32, sr[j]);
             ptx::tmem_wait_ld();
-            if (nvalid < T::BN) {
+            if (c_lo > 0 || c_hi < T::BN) {
 #pragma unroll
               for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int c = 0; c < 32; ++c)
-                  if (j * 32 + c >= nvalid) sr[j][c] = __float_as_uint(-INFINITY);
+                  if (j * 32 + c < c_lo || j * 32 + c >= c_hi)
+                    sr[j][c] = __float_as_uint(-INFINITY);
             }
             // Row max as a tree over 8 independent running maxima (3-input max).
             float mx8[8];
@@ -598,7 +648,9 @@ __global__ void __launch_bounds__(384, 1)
             float rs8[8];
 #pragma unroll
             for (int a = 0; a < 8; ++a) rs8[a] = 0.f;
-            const float sl = p.scale_log2, nm = -m;
+            // A row of a frame-aligned unit can meet a source tile wholly outside its
+            // frame before any visible key (m still -inf): subtract 0 there, not -inf.
+            const float sl = p.scale_log2, nm = (kAligned && m == -INFINITY) ? 0.f : -m;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               uint32_t pk[16];
@@ -649,7 +701,7 @@ __global__ void __launch_bounds__(384, 1)
             const int nu = next_visited(mo, mo1, gstart[g] + t + 1, gstart[ghi]);
             if (nu < gstart[ghi] && nu >= gstart[g + 1])
               while (gn + 1 < ghi && nu >= gstart[gn + 1]) ++gn;
-          } else if (t == nkt - 1 && g + 1 < ghi) {
+          } else if (t == t1 - 1 && g + 1 < ghi) {
             gn = g + 1;
           }
           if (gn != g) {

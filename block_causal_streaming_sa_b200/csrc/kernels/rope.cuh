@@ -68,7 +68,7 @@ __device__ __forceinline__ void st_v4(void* p, uint4 v) {
 
 // One block per token (b, l); thread t moves 16-byte chunk t % (D/8) of head
 // t / (D/8). blockIdx.y: 0 = K (bf16 in, rotated, fp16 out), 1 = V (bf16,
-// copied). Loads are fully coalesced (a token's H*D values are contiguous); each head's 2*D bytes are
+// copied; rotated like K when second_is_key). Loads are fully coalesced (a token's H*D values are contiguous); each head's 2*D bytes are
 // stored contiguously into its [B, H, L_out, D] plane.
 __global__ void rope_transpose_kernel(AppendParams p) {
   const int vec_per_head = p.D >> 3;
@@ -84,7 +84,7 @@ __global__ void rope_transpose_kernel(AppendParams p) {
   const size_t src = (static_cast<size_t>(tok) * p.H + h) * p.D + c * 8;
   const size_t dst = ((static_cast<size_t>(b) * p.H + h) * p.L_out + l) * p.D + c * 8;
   uint4 v = ld_nc_v4(in + src);
-  if (!is_v) {
+  if (!is_v || p.second_is_key) {
     const int f = l / p.rope.frame_tokens;
     const int y = (l / p.rope.tok_w) % p.rope.tok_h;
     const int x = l % p.rope.tok_w;

@@ -115,8 +115,8 @@ Derived derive(const sa_config& c) {
     d.off_tier[t] = off;
     off += align_up(static_cast<size_t>(d.S + d.R) * slot_bytes, 1024);
   }
-  d.off_kcur = off;
-  off += align_up(d.chunk_elems * sizeof(__nv_bfloat16), 1024);
+  d.off_kcur = off;  // [target | source] rotated keys of the generating chunk
+  off += align_up(2 * d.chunk_elems * sizeof(__nv_bfloat16), 1024);
   d.off_ref = off;
   off += align_up(2 * d.ref_elems * sizeof(__nv_bfloat16), 1024);
   // split-tail scratch: partial rows, their lse, per-row merge counters
@@ -212,42 +212,59 @@ unsigned attend_grid(const Derived& d, int rows, int sm_count, bool split_ok) {
 }
 
 // The attention kernel instantiations: head dim 128 / 64, dense / block-sparse.
-// Tensor maps of one launch: cache tier, key scratch, current V, reference.
+// Tensor maps of one launch: cache tier, key scratch, current V, reference,
+// source V (frame-aligned editing).
 struct AttendMaps {
   const CUtensorMap* cache;
   const CUtensorMap* kcur;
   const CUtensorMap* vcur;
   const CUtensorMap* ref;
+  const CUtensorMap* vsrc;
 };
 
-template <int D, bool kSparse>
+template <int D, int kMode>
 void launch_attend_tc_t(unsigned grid, cudaStream_t s, const AttendMaps& m,
                         const AttendParams& ap) {
-  sa::attend_tc_kernel<D, kSparse><<<grid, sa::TcShape<D>::kThreads, sa::TcShape<D>::kSmemBytes,
-                                     s>>>(*m.cache, *m.kcur, *m.vcur, *m.ref, ap);
+  sa::attend_tc_kernel<D, kMode><<<grid, sa::TcShape<D>::kThreads, sa::TcShape<D>::kSmemBytes,
+                                   s>>>(*m.cache, *m.kcur, *m.vcur, *m.ref, *m.vsrc, ap);
 }
 
-void launch_attend_tc(int D, bool sparse, unsigned grid, cudaStream_t s, const AttendMaps& m,
+template <int D>
+void launch_attend_tc_d(int mode, unsigned grid, cudaStream_t s, const AttendMaps& m,
+                        const AttendParams& ap) {
+  if (mode == sa::kModeSparse)
+    launch_attend_tc_t<D, sa::kModeSparse>(grid, s, m, ap);
+  else if (mode == sa::kModeAligned)
+    launch_attend_tc_t<D, sa::kModeAligned>(grid, s, m, ap);
+  else
+    launch_attend_tc_t<D, sa::kModeDense>(grid, s, m, ap);
+}
+
+void launch_attend_tc(int D, int mode, unsigned grid, cudaStream_t s, const AttendMaps& m,
                       const AttendParams& ap) {
   if (D == 128)
-    sparse ? launch_attend_tc_t<128, true>(grid, s, m, ap)
-           : launch_attend_tc_t<128, false>(grid, s, m, ap);
+    launch_attend_tc_d<128>(mode, grid, s, m, ap);
   else
-    sparse ? launch_attend_tc_t<64, true>(grid, s, m, ap)
-           : launch_attend_tc_t<64, false>(grid, s, m, ap);
+    launch_attend_tc_d<64>(mode, grid, s, m, ap);
 }
 
 // Every instantiation: the register count the setmaxnreg split assumes, and the
 // dynamic shared memory it needs.
-template <int D, bool kSparse>
+template <int D, int kMode>
 bool prepare_attend_tc_t() {
   cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, sa::attend_tc_kernel<D, kSparse>) != cudaSuccess ||
+  if (cudaFuncGetAttributes(&fa, sa::attend_tc_kernel<D, kMode>) != cudaSuccess ||
       fa.numRegs != sa::TcShape<D>::kLaunchRegs)
     return false;
-  return cudaFuncSetAttribute(sa::attend_tc_kernel<D, kSparse>,
+  return cudaFuncSetAttribute(sa::attend_tc_kernel<D, kMode>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               sa::TcShape<D>::kSmemBytes) == cudaSuccess;
+}
+
+template <int D>
+bool prepare_attend_tc_d() {
+  return prepare_attend_tc_t<D, sa::kModeDense>() && prepare_attend_tc_t<D, sa::kModeSparse>() &&
+         prepare_attend_tc_t<D, sa::kModeAligned>();
 }
 
 __global__ void exp2_probe_kernel(const float* x, float* y, int n, int poly) {
@@ -267,6 +284,7 @@ struct sa_handle {
   int frames[2][SA_MAX_ATTENDED];  // frames of the chunk each slot holds, per tier
   int staged_chunk;                // chunk whose keys sit in the scratch (-1: none)
   int staged_frames;               // its frames
+  bool staged_source;              // source-frame keys staged beside them
   bool has_cache;
   bool has_ref;  // a reference image is set
   CUtensorMap tm_tier[2];
@@ -307,9 +325,11 @@ int check_device(sa_handle* h) {
   return SA_OK;
 }
 
-// Rotate K (and copy V, if given) of `rows` tokens into [B, H, L_out, D] planes.
+// Rotate K (and copy V, if given; rotate it too with second_is_key) of `rows`
+// tokens into [B, H, L_out, D] planes.
 int launch_rope_transpose(sa_handle* h, const void* K, const void* V, __nv_bfloat16* k_out,
-                          __nv_bfloat16* v_out, int rows, int L_out, cudaStream_t s) {
+                          __nv_bfloat16* v_out, int rows, int L_out, cudaStream_t s,
+                          bool second_is_key = false) {
   const Derived& d = h->d;
   AppendParams ap;
   ap.k_in = static_cast<const __nv_bfloat16*>(K);
@@ -321,6 +341,7 @@ int launch_rope_transpose(sa_handle* h, const void* K, const void* V, __nv_bfloa
   ap.H = d.H;
   ap.D = d.D;
   ap.L_out = L_out;
+  ap.second_is_key = second_is_key ? 1 : 0;
   ap.rope = h->rope();
   const int threads = static_cast<int>(align_up(static_cast<size_t>(d.H) * d.D / 8, 32));
   dim3 grid(static_cast<unsigned>(d.B) * rows, V != nullptr ? 2 : 1);
@@ -371,9 +392,11 @@ Plan make_plan(const sa_handle* h, int tier, int n_frames) {
   return pl;
 }
 
-// Key groups of the attention kernels: the reference image (if set), then the
-// plan's chunks. t_delta = base(current) - base(group) >= 0.
-void fill_groups(const sa_handle* h, int tier, int n_frames, AttendParams* ap) {
+// Key groups of the attention kernels: the reference image (if set), the plan's
+// chunks, and for frame-aligned editing the source frames of the generating
+// chunk (same positions as its own frames: t_delta 0). t_delta = base(current) -
+// base(group) >= 0.
+void fill_groups(const sa_handle* h, int tier, int n_frames, bool source, AttendParams* ap) {
   const Derived& d = h->d;
   const Plan pl = make_plan(h, tier, n_frames);
   const int base_c = pl.base[pl.n - 1];
@@ -392,12 +415,25 @@ void fill_groups(const sa_handle* h, int tier, int n_frames, AttendParams* ap) {
     grp.t_delta = base_c - pl.base[g];
     grp.len = pl.frames[g] * d.th * d.tw;
   }
+  if (source) {
+    AttendGroup& grp = ap->groups[n++];
+    grp.src = 3;
+    grp.slot = 0;
+    grp.t_delta = 0;
+    grp.len = n_frames * d.th * d.tw;
+  }
   ap->n_groups = n;
 }
 
+// Most key groups an attention of this config can have (the kernel's table holds
+// kMaxGroups): S + W chunks, the reference, the source frames.
+int max_groups(const sa_handle* h, bool source) {
+  return h->d.S + h->d.W + (h->d.RF > 0 ? 1 : 0) + (source ? 1 : 0);
+}
+
 // Everything of AttendParams but the key source of the current chunk.
-void fill_common(sa_handle* h, int tier, int n_frames, const void* Q, const void* Vc, void* O,
-                 float* lse, AttendParams* ap) {
+void fill_common(sa_handle* h, int tier, int n_frames, bool source, const void* Q,
+                 const void* Vc, void* O, float* lse, AttendParams* ap) {
   const Derived& d = h->d;
   std::memset(ap, 0, sizeof(*ap));
   ap->q = static_cast<const __nv_bfloat16*>(Q);
@@ -412,7 +448,7 @@ void fill_common(sa_handle* h, int tier, int n_frames, const void* Q, const void
   ap->D = d.D;
   ap->L_plane = d.L;
   ap->L_ref = d.Lref;
-  fill_groups(h, tier, n_frames, ap);
+  fill_groups(h, tier, n_frames, source, ap);
   ap->scale_log2 = d.scale * 1.4426950408889634f;
   ap->rope = h->rope();
   ap->status = h->status();
@@ -430,38 +466,57 @@ int check_attend_ptrs(sa_handle* h, const void* Q, const void* Vc, const void* O
   return SA_OK;
 }
 
-int stage_keys(sa_handle* h, const void* Kc, int n_frames, sa_stream stream) {
+// Rotate the generating chunk's keys (and, for frame-aligned editing, its
+// source keys Ks) into the key scratch.
+int stage_keys(sa_handle* h, const void* Kc, int n_frames, sa_stream stream,
+               const void* Ks = nullptr) {
   int rc = check_handle(h);
   if (rc != SA_OK) return rc;
   rc = check_frames(h, n_frames);
   if (rc != SA_OK) return rc;
   if (Kc == nullptr || !aligned16(Kc))
     return h->fail(SA_ERR_INVALID_ARG, "Kc must be a non-NULL 16-byte aligned pointer");
+  if (Ks != nullptr && !aligned16(Ks))
+    return h->fail(SA_ERR_INVALID_ARG, "Ks must be 16-byte aligned");
   if (h->count[0] != h->count[1])
     return h->fail(SA_ERR_STATE, "both tiers must hold the same chunks before attending");
   rc = check_device(h);
   if (rc != SA_OK) return rc;
-  rc = launch_rope_transpose(h, Kc, nullptr, h->kcur(), nullptr, n_frames * h->d.th * h->d.tw,
-                             h->d.L, reinterpret_cast<cudaStream_t>(stream));
+  rc = launch_rope_transpose(h, Kc, Ks, h->kcur(), h->kcur() + h->d.chunk_elems,
+                             n_frames * h->d.th * h->d.tw, h->d.L,
+                             reinterpret_cast<cudaStream_t>(stream), Ks != nullptr);
   if (rc != SA_OK) return rc;
   h->staged_chunk = h->count[0];
   h->staged_frames = n_frames;
+  h->staged_source = Ks != nullptr;
   return SA_OK;
 }
 
+// The attention launch over the staged keys. Vs non-null: frame-aligned editing
+// (the source keys must have been staged with the chunk's keys).
 int attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final, void* O,
                   float* lse, sa_stream stream, bool simt, bool debug_stall = false,
-                  const uint8_t* block_mask = nullptr) {
+                  const uint8_t* block_mask = nullptr, const void* Vs = nullptr) {
   int rc = check_handle(h);
   if (rc != SA_OK) return rc;
   rc = check_attend_ptrs(h, Q, Vc, O, lse);
   if (rc != SA_OK) return rc;
+  const bool aligned = Vs != nullptr;
+  if (aligned && (!aligned16(Vs) || O == Vs))
+    return h->fail(SA_ERR_INVALID_ARG, "Vs must be 16-byte aligned and not aliased by O");
+  if (aligned && !h->staged_source)
+    return h->fail(SA_ERR_STATE, "no source keys staged for frame-aligned attention");
+  if (aligned && (simt || block_mask != nullptr))
+    return h->fail(SA_ERR_UNSUPPORTED, "frame-aligned attention runs on the dense kernel only");
   if (h->count[0] != h->count[1])
     return h->fail(SA_ERR_STATE, "both tiers must hold the same chunks before attending");
   if (h->staged_chunk != h->count[0])
     return h->fail(SA_ERR_STATE, "no keys staged for the current chunk (call sa_stage_keys)");
   if (block_mask != nullptr && h->has_ref)
     return h->fail(SA_ERR_UNSUPPORTED, "block-sparse attention takes no reference image");
+  if (max_groups(h, aligned) > sa::kMaxGroups)
+    return h->fail(SA_ERR_UNSUPPORTED, "more than SA_MAX_ATTENDED key groups (chunks, "
+                                       "reference and source frames)");
   rc = check_device(h);
   if (rc != SA_OK) return rc;
   const Derived& d = h->d;
@@ -469,7 +524,7 @@ int attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final
   const int tier = step_is_final ? SA_TIER_CLEAN : SA_TIER_NOISY;
 
   AttendParams ap;
-  fill_common(h, tier, h->staged_frames, Q, Vc, O, lse, &ap);
+  fill_common(h, tier, h->staged_frames, aligned, Q, Vc, O, lse, &ap);
   ap.k_cur = h->kcur();
   ap.debug_stall_producer = debug_stall ? 1 : 0;
   ap.block_mask = block_mask;
@@ -486,12 +541,16 @@ int attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final
     else
       sa::attend_simt_kernel<64><<<grid, 256, 0, s>>>(ap);
   } else {
-    CUtensorMap tm_v;
-    if (!encode_blhd(&tm_v, Vc, d, ap.L)) return h->fail(SA_ERR_CUDA, "TMA descriptor for Vc failed");
+    CUtensorMap tm_v, tm_vs;
+    if (!encode_blhd(&tm_v, Vc, d, ap.L) || (aligned && !encode_blhd(&tm_vs, Vs, d, ap.L)))
+      return h->fail(SA_ERR_CUDA, "TMA descriptor for Vc / Vs failed");
     AttendMaps maps{h->has_cache ? &h->tm_tier[tier] : &h->tm_kcur, &h->tm_kcur, &tm_v,
-                    d.RF > 0 ? &h->tm_ref : &h->tm_kcur};
-    launch_attend_tc(d.D, block_mask != nullptr,
-                     attend_grid(d, ap.L, h->sm_count, ap.split_ok != 0), s, maps, ap);
+                    d.RF > 0 ? &h->tm_ref : &h->tm_kcur, aligned ? &tm_vs : &tm_v};
+    const int mode = block_mask != nullptr ? sa::kModeSparse
+                     : aligned             ? sa::kModeAligned
+                                           : sa::kModeDense;
+    launch_attend_tc(d.D, mode, attend_grid(d, ap.L, h->sm_count, ap.split_ok != 0), s, maps,
+                     ap);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
@@ -514,6 +573,28 @@ int attend_common(sa_handle* h, const void* Q, const void* Kc, const void* Vc, i
   rc = stage_keys(h, Kc, n_frames, stream);
   if (rc != SA_OK) return rc;
   return attend_staged(h, Q, Vc, step_is_final, O, lse, stream, simt, false, block_mask);
+}
+
+int attend_aligned(sa_handle* h, const void* Q, const void* Kc, const void* Vc, const void* Ks,
+                   const void* Vs, int n_frames, int step_is_final, void* O, float* lse,
+                   sa_stream stream) {
+  int rc = check_handle(h);
+  if (rc != SA_OK) return rc;
+  if (Kc == nullptr || Ks == nullptr || Vs == nullptr)
+    return h->fail(SA_ERR_INVALID_ARG, "Kc, Ks and Vs must be non-NULL");
+  if (!aligned16(Ks) || !aligned16(Vs))
+    return h->fail(SA_ERR_INVALID_ARG, "Ks and Vs must be 16-byte aligned");
+  if (O == Kc || O == Ks || O == Vs)
+    return h->fail(SA_ERR_INVALID_ARG, "O must not alias an input");
+  // Validate the attention half before launching the staging half.
+  rc = check_attend_ptrs(h, Q, Vc, O, lse);
+  if (rc != SA_OK) return rc;
+  if (max_groups(h, true) > sa::kMaxGroups)
+    return h->fail(SA_ERR_UNSUPPORTED, "more than SA_MAX_ATTENDED key groups (chunks, "
+                                       "reference and source frames)");
+  rc = stage_keys(h, Kc, n_frames, stream, Ks);
+  if (rc != SA_OK) return rc;
+  return attend_staged(h, Q, Vc, step_is_final, O, lse, stream, false, false, nullptr, Vs);
 }
 
 // ---------------------------------------------------------------- sa_attend_noalloc
@@ -571,7 +652,7 @@ int attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc, 
     return h->fail(SA_ERR_CUDA, "TMA descriptors for sa_attend_noalloc failed");
 
   AttendParams ap;
-  fill_common(h, tier, d.F, Q, Vc, O, lse, &ap);
+  fill_common(h, tier, d.F, false, Q, Vc, O, lse, &ap);
   ap.k_cur = keys;
   ap.split_ok = 0;  // no scratch but the fixed key array: no split tail
 
@@ -580,8 +661,8 @@ int attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc, 
   rc = launch_rope_transpose(h, Kc, nullptr, keys, nullptr, d.L, d.L, s);
   if (rc != SA_OK) return rc;
   AttendMaps maps{h->has_cache ? &h->tm_tier[tier] : &tm_keys, &tm_keys, &tm_v,
-                  d.RF > 0 ? &h->tm_ref : &tm_keys};
-  launch_attend_tc(d.D, false, attend_grid(d, d.L, h->sm_count, false), s, maps, ap);
+                  d.RF > 0 ? &h->tm_ref : &tm_keys, &tm_v};
+  launch_attend_tc(d.D, sa::kModeDense, attend_grid(d, d.L, h->sm_count, false), s, maps, ap);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
     return h->fail(SA_ERR_CUDA, std::string("attend launch: ") + cudaGetErrorString(e));
@@ -699,6 +780,7 @@ SA_API int sa_create(const sa_config* cfg, void* dev_buf, size_t bytes, sa_handl
     for (int s = 0; s < SA_MAX_ATTENDED; ++s) h->frames[t][s] = d.F;
   h->staged_chunk = -1;
   h->staged_frames = d.F;
+  h->staged_source = false;
   h->has_ref = false;
 
   // RoPE tables: angle pos * theta^(-2i/d) in double, cos/sin cast to float.
@@ -741,7 +823,7 @@ SA_API int sa_create(const sa_config* cfg, void* dev_buf, size_t bytes, sa_handl
         return SA_ERR_CUDA;
       }
   }
-  if (!encode_planes(&h->tm_kcur, h->kcur(), d, d.L, 1LL * d.B * d.H)) {
+  if (!encode_planes(&h->tm_kcur, h->kcur(), d, d.L, 2LL * d.B * d.H)) {
     g_error = "TMA descriptor for the key scratch failed";
     delete h;
     return SA_ERR_CUDA;
@@ -753,8 +835,7 @@ SA_API int sa_create(const sa_config* cfg, void* dev_buf, size_t bytes, sa_handl
   }
   // The kernel's register split assumes it is launched with exactly
   // TcShape::kLaunchRegs registers per thread; refuse to run otherwise.
-  if (!prepare_attend_tc_t<128, false>() || !prepare_attend_tc_t<128, true>() ||
-      !prepare_attend_tc_t<64, false>() || !prepare_attend_tc_t<64, true>()) {
+  if (!prepare_attend_tc_d<128>() || !prepare_attend_tc_d<64>()) {
     g_error = "attention kernel: unexpected register count or shared memory attribute failed";
     delete h;
     return SA_ERR_UNSUPPORTED;
@@ -828,6 +909,12 @@ SA_API int sa_attend_frames(sa_handle* h, const void* Q, const void* Kc, const v
                             int n_frames, int step_is_final, void* O, float* lse,
                             sa_stream stream) {
   return attend_common(h, Q, Kc, Vc, n_frames, step_is_final, O, lse, stream, false);
+}
+
+SA_API int sa_attend_aligned(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
+                             const void* Ks, const void* Vs, int n_frames, int step_is_final,
+                             void* O, float* lse, sa_stream stream) {
+  return attend_aligned(h, Q, Kc, Vc, Ks, Vs, n_frames, step_is_final, O, lse, stream);
 }
 
 SA_API int sa_stage_keys(sa_handle* h, const void* Kc, sa_stream stream) {

@@ -12,6 +12,13 @@ namespace sa {
 constexpr int kMaxGroups = SA_MAX_ATTENDED;
 constexpr int kMaxSplitSlots = 128;  // tail tiles that may be split (grids of up to 256 CTAs)
 
+// Attention kernel variants: every attended key (dense), caller-flagged 128 x 128
+// blocks (sparse), or dense plus a last key group of source frames each query row
+// sees only its own frame of (frame-aligned editing).
+constexpr int kModeDense = 0;
+constexpr int kModeSparse = 1;
+constexpr int kModeAligned = 2;
+
 // Device status word bits (written with atomicOr, read by sa_get_status).
 constexpr unsigned kDevErrTimeout = 1u;
 
@@ -29,7 +36,8 @@ struct RopeTables {
 // Rotate-and-transpose of one chunk (or the reference image): in [B, L, H, D]
 // -> out [B, H, L_out, D] (planes of L_out >= L rows; rows L.. untouched).
 // K rows (bf16) are turned by their in-chunk (frame, row, column) position and
-// written as fp16; V rows (blockIdx.y == 1) are copied as bf16.
+// written as fp16; V rows (blockIdx.y == 1) are copied as bf16, or, with
+// second_is_key, turned and written as fp16 like K (two key tensors at once).
 struct AppendParams {
   const __nv_bfloat16* k_in;
   const __nv_bfloat16* v_in;  // may be null (K only)
@@ -37,6 +45,7 @@ struct AppendParams {
   __nv_bfloat16* v_out;
   int B, L, H, D;
   int L_out;  // rows per output plane
+  int second_is_key;
   RopeTables rope;
 };
 
@@ -44,7 +53,8 @@ struct AppendParams {
 // attended chunks in ascending chunk-id order.
 struct AttendGroup {
   int src;      // 0: cache slot of the selected tier, 1: the chunk being generated,
-                // 2: the reference image
+                // 2: the reference image, 3: the source frames of the chunk being
+                // generated (frame-aligned editing; always the last group)
   int slot;     // cache slot (src == 0)
   int t_delta;  // temporal base of the current chunk minus this group's, >= 0
   int len;      // number of keys
@@ -57,7 +67,8 @@ struct AttendParams {
   const __nv_bfloat16* cache;    // selected tier: [slot][K|V][B][H][L_plane][D]; K planes
                                  // hold fp16 keys rotated in-chunk, V planes bf16
   const __nv_bfloat16* k_cur;    // current chunk K (fp16 bits), rotated in-chunk:
-                                 // [B][H][L_plane][D]
+                                 // [B][H][L_plane][D]; for frame-aligned editing the
+                                 // source keys follow as a second [B][H][L_plane][D]
   const __nv_bfloat16* v_cur;    // current chunk V as passed: [B][L][H][D]
   const __nv_bfloat16* ref;      // reference image [K|V][B][H][L_ref][D] (K fp16) or null
   int B, L, H, D;                // L: query rows of the current chunk

@@ -109,6 +109,26 @@ class StreamingAttention:
                                lse_ptr, self._stream(stream))
         return out
 
+    def attend_aligned(self, Q, Kc, Vc, Ks, Vs, step_is_final, out=None, lse=None, stream=None):
+        """Frame-aligned editing attention: the usual keys plus, for each query
+        token, the source tokens Ks/Vs of its own frame (same shape as Q)."""
+        n = self._frames_of(Q, "Q")
+        shape = self._shape(n)
+        if out is None:
+            out = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
+        lse_ptr = 0
+        if lse is not None:
+            b, l, h, _ = shape
+            if lse.dtype != torch.float32 or tuple(lse.shape) != (b, h, l) \
+                    or not lse.is_contiguous():
+                raise ValueError(f"lse must be contiguous fp32 of shape {(b, h, l)}")
+            lse_ptr = lse.data_ptr()
+        ptrs = [self._ptr(t, name, n) for t, name in
+                ((Q, "Q"), (Kc, "Kc"), (Vc, "Vc"), (Ks, "Ks"), (Vs, "Vs"))]
+        B.sa_attend_aligned(self.handle, *ptrs, n, step_is_final, self._ptr(out, "O", n), lse_ptr,
+                            self._stream(stream))
+        return out
+
     def plan(self, step_is_final, n_frames=None):
         """(ids, t_base, lens) the next attention would use."""
         return B.sa_stream_plan(self.handle, step_is_final,

@@ -87,8 +87,9 @@ SA_API int sa_validate_config(const sa_config* cfg);
 
 /* Bytes of device memory sa_create needs for cfg (0 if cfg is invalid):
  * a status word, fp32 RoPE tables, both cache tiers ((S + W - 1) slots of K and
- * V each, layout [slot][K|V][B][H][L][D], K fp16, V bf16), one rotated-key chunk of scratch
- * for the chunk being generated and, when ref_frames > 0, the reference image
+ * V each, layout [slot][K|V][B][H][L][D], K fp16, V bf16), two rotated-key chunks of
+ * scratch for the chunk being generated (its keys and, for sa_attend_aligned,
+ * its source keys) and, when ref_frames > 0, the reference image
  * ([K|V][B][H][ref_frames * tok_h * tok_w][D]). Host only. */
 SA_API size_t sa_required_bytes(const sa_config* cfg);
 
@@ -170,6 +171,26 @@ SA_API int sa_attend(sa_handle* h, const void* Q, const void* Kc, const void* Vc
 SA_API int sa_attend_frames(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
                             int n_frames, int step_is_final, void* O, float* lse,
                             sa_stream stream);
+
+/* Frame-aligned editing attention. "Vidu S2：实时可交互、可编辑、可立体的视频生成",
+ * section 2.6 (the editing model S2-Editing): the source video is encoded as
+ * condition tokens next to the noisy target tokens; every generated frame
+ * exchanges information only with the source frame of the same moment; the
+ * reference image is seen by every frame; each source frame is consumed with
+ * its target frame and never cached ("Vidu S2：实时数字人、实时视频编辑都做到了，空间视频还只是
+ * 探索", section on S2-Editing, says the same).
+ * Computes sa_attend_frames over the usual keys (reference if set, cached sink
+ * and window chunks of the selected tier, the chunk's own Kc/Vc) plus the
+ * source tokens Ks/Vs ([B, Lc, H, D] bf16, unrotated, the same frames and
+ * token grid as Q), where a query token of frame f sees only the source tokens
+ * of frame f. Source frame f takes the temporal and spatial coordinates of
+ * target frame f. Nothing of Ks/Vs is kept after the call. The key scratch
+ * holds Kc and Ks rotated; one staging launch and one attention launch.
+ * Needs S + W (+ 1 with a reference) + 1 <= SA_MAX_ATTENDED key groups, else
+ * SA_ERR_UNSUPPORTED. O, lse, n_frames and the error rules as sa_attend_frames. */
+SA_API int sa_attend_aligned(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
+                             const void* Ks, const void* Vs, int n_frames, int step_is_final,
+                             void* O, float* lse, sa_stream stream);
 
 /* Block-sparse attention ("Vidu S2 vs PixVerse R2：实时视频的两条技术路线", section
  * 选择四：速度从哪里来: PixVerse R2 learns block-sparse attention and skips more than
