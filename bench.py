@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--sparsity", type=float, default=0.0,
                     help="block-sparse mode: share of 128x128 blocks skipped (seeded random mask)")
+    ap.add_argument("--ulysses", action="store_true",
+                    help="head-sharded attention over the ranks (Ulysses, fp8 exchange)")
     ap.add_argument("--editing", action="store_true",
                     help="frame-aligned editing attention (source frames of the chunk as extra keys)")
     ap.add_argument("--ref-frames", type=int, default=0,
@@ -312,15 +314,28 @@ def run_ours(args, w):
 
     stream = torch.cuda.Stream(device=dev)
     names = ("Q", "Kc", "Vc", "Kn", "Vn", "Kcl", "Vcl") + (("Ks", "Vs") if args.editing else ())
-    pool_host = [{n: w.tensor(n, 100 + c, layer=rank).pin_memory() for n in names}
-                 for c in range(2)]
+    shard = slice(None)
+    if args.ulysses:
+        # Ulysses: every rank holds 1/N of each chunk's tokens with all heads
+        if w.chunk_len % world or w.heads % world:
+            raise SystemExit("--ulysses needs tokens and heads divisible by the rank count")
+        t = w.chunk_len // world
+        shard = slice(rank * t, (rank + 1) * t)
+    pool_host = [{n: w.tensor(n, 100 + c, layer=0 if args.ulysses else rank)[:, shard]
+                  .contiguous().pin_memory() for n in names} for c in range(2)]
     pool = [{n: t.to(dev) for n, t in s.items()} for s in pool_host]
-    out = torch.empty(w.shape(), dtype=torch.bfloat16, device=dev)
-    out_host = torch.empty(w.shape(), dtype=torch.bfloat16).pin_memory()
+    out_shape = tuple(pool[0]["Q"].shape)
+    out = torch.empty(out_shape, dtype=torch.bfloat16, device=dev)
+    out_host = torch.empty(out_shape, dtype=torch.bfloat16).pin_memory()
 
     # One handle (its own two-tier cache) per attention layer of the workload.
     cfg = dict(w.config_dict(), ref_frames=args.ref_frames)
-    layers = [sa.StreamingAttention(cfg, device=dev) for _ in range(w.layers)]
+    if args.ulysses:
+        from block_causal_streaming_sa_b200.ulysses import UlyssesAttention
+
+        layers = [UlyssesAttention(cfg, device=dev) for _ in range(w.layers)]
+    else:
+        layers = [sa.StreamingAttention(cfg, device=dev) for _ in range(w.layers)]
     attn = layers[0]
     sp = stream.cuda_stream
     flops = attend_flops(w)
@@ -329,8 +344,12 @@ def run_ours(args, w):
         # A reference image of ref_frames frames, set once (its keys are rotated
         # on the way in); every attention also reads its ref_len keys.
         ref_shape = (w.batch, ref_len, w.heads, w.head_dim)
-        Kref, Vref = (normal_bf16(seed_of(w.name, "reference", n), ref_shape).to(dev)
-                      for n in ("K", "V"))
+        ref_shard = slice(None)
+        if args.ulysses:
+            t = ref_len // world
+            ref_shard = slice(rank * t, (rank + 1) * t)
+        Kref, Vref = (normal_bf16(seed_of(w.name, "reference", n), ref_shape)[:, ref_shard]
+                      .contiguous().to(dev) for n in ("K", "V"))
         for layer in layers:
             layer.set_reference(Kref, Vref)
         torch.cuda.synchronize(dev)
@@ -343,6 +362,11 @@ def run_ours(args, w):
     appends_per_chunk = 2 * w.layers
 
     def append_all(s):
+        if args.ulysses:
+            for layer in layers:
+                layer.append(sa.SA_TIER_NOISY, s["Kn"], s["Vn"])
+                layer.append(sa.SA_TIER_CLEAN, s["Kcl"], s["Vcl"])
+            return
         for layer in layers:
             h = layer.handle
             sa.sa_append_chunk(h, sa.SA_TIER_NOISY, s["Kn"].data_ptr(), s["Vn"].data_ptr(), sp)
@@ -363,12 +387,23 @@ def run_ours(args, w):
                                           * keys[None, :].double()).sum())
         block_mask = block_mask.to(torch.uint8).to(dev)
 
+    res = [out]  # the last attention output (the Ulysses layer returns its own tensor)
+
     def chunk_step(s, ev=None):
         """One chunk: every denoising step's attention in every layer, then the appends."""
         a = 0
         for k in range(steps_per_chunk):
             final = k == steps_per_chunk - 1
             for layer in layers:
+                if args.ulysses:
+                    # the whole layer call: exchanges in, attention, exchange out
+                    if ev is not None:
+                        ev[0][a].record(stream)
+                    res[0] = layer.attend(s["Q"], s["Kc"], s["Vc"], final)
+                    if ev is not None:
+                        ev[1][a].record(stream)
+                    a += 1
+                    continue
                 h = layer.handle
                 if args.editing:
                     # editing: the staging of Kc and Ks is inside the timed call
@@ -438,7 +473,7 @@ def run_ours(args, w):
             for n, t in pool_host[i % 2].items():
                 dev_bufs[n].copy_(t, non_blocking=True)
             chunk_step(dev_bufs)
-            out_host.copy_(out, non_blocking=True)
+            out_host.copy_(res[0], non_blocking=True)
         stream.synchronize()
         barrier()
         e0, e1 = mk(), mk()
@@ -447,7 +482,7 @@ def run_ours(args, w):
             for n, t in pool_host[i % 2].items():
                 dev_bufs[n].copy_(t, non_blocking=True)
             chunk_step(dev_bufs)
-            out_host.copy_(out, non_blocking=True)
+            out_host.copy_(res[0], non_blocking=True)
         e1.record(stream)
         stream.synchronize()
         e2e_ms_local = e0.elapsed_time(e1)
@@ -455,8 +490,11 @@ def run_ours(args, w):
 
     ms_max = max_over_ranks(ms_local)
     e2e_ms_max = max_over_ranks(e2e_ms_local)
-    value = whole_job_tflops(flops * attends_per_chunk * args.steps, ms_max, world)
-    e2e_value = whole_job_tflops(flops * attends_per_chunk * e2e_steps, e2e_ms_max, world)
+    # Ulysses splits one layer's attention over the ranks (strong scaling): each
+    # rank does 1/world of it; replicas each do a whole one (weak scaling).
+    flops_rank = flops / world if args.ulysses else flops
+    value = whole_job_tflops(flops_rank * attends_per_chunk * args.steps, ms_max, world)
+    e2e_value = whole_job_tflops(flops_rank * attends_per_chunk * e2e_steps, e2e_ms_max, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -468,7 +506,7 @@ def run_ours(args, w):
 
     peaks, peak_src = load_peaks()
     attend_avg = statistics.fmean(attend_ms)
-    achieved = flops / (attend_avg * 1e-3) / 1e12
+    achieved = flops_rank / (attend_avg * 1e-3) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     append_bytes = appends_per_chunk * 2 * 2 * (w.batch * w.chunk_len * w.heads * w.head_dim * 2)
@@ -484,7 +522,7 @@ def run_ours(args, w):
         "warmup": args.warmup,
         "ms_per_step": ms_max / args.steps,
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if args.ulysses else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
@@ -495,7 +533,8 @@ def run_ours(args, w):
             "step": "all denoising attentions of one chunk (every layer) + noisy and clean appends",
             "l2": f"inputs larger than L2: {cache_bytes_read / 2**20:.0f} MiB of cached K/V "
                   f"read per attention vs {L2_BYTES / 2**20:.0f} MiB L2",
-            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "parallelism": (f"ulysses{world}" if args.ulysses else
+                            f"replicas{world}" if world > 1 else "single"),
             "block_sparsity": args.sparsity,
             "ref_frames": args.ref_frames, "ref_tokens": ref_len,
             "frame_aligned_editing": args.editing,
@@ -503,6 +542,8 @@ def run_ours(args, w):
         "roofline": {
             "bound": "tensor",
             "kernel": "attend_tc_kernel<128>" + (
+                " (Ulysses layer call: fp8 pack, all-to-all, staging, attention, unpack)"
+                if args.ulysses else
                 " (sparse, timed with its staging kernel)" if block_mask is not None else
                 " (frame-aligned, timed with its staging kernel)" if args.editing else ""),
             "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
@@ -516,7 +557,10 @@ def run_ours(args, w):
         "attention_tflops_kernel": achieved,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms_max / e2e_steps},
-        "gpu_launches": args.steps * (2 * attends_per_chunk + appends_per_chunk),
+        # per attention: stage + attend (+ 4 pack/unpack pairs with Ulysses);
+        # per append: one kernel (+ 2 pack/unpack pairs with Ulysses)
+        "gpu_launches": args.steps * ((10 if args.ulysses else 2) * attends_per_chunk
+                                      + (5 if args.ulysses else 1) * appends_per_chunk),
         "clocks": clock_info,
         "cpu_baseline": cpu,
     }

@@ -24,6 +24,8 @@ SA_TIER_NOISY = 0
 SA_TIER_CLEAN = 1
 SA_MAX_ATTENDED = 16
 SA_NOALLOC_MAX_KEY_BYTES = 64 << 20
+SA_PAYLOAD_FP8 = 0
+SA_PAYLOAD_BF16 = 1
 
 
 class SaConfig(ctypes.Structure):
@@ -80,6 +82,9 @@ _SIGNATURES = {
     "sa_plan": (_I, [_CFGP, ctypes.c_int32, _I32P, _I32P, _I32P, _I]),
     "sa_stream_plan": (_I, [_P, _I, _I, _I32P, _I32P, _I32P, _I]),
     "sa_slot_of": (_I, [_CFGP, ctypes.c_int32]),
+    "sa_exchange_block_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I]),
+    "sa_exchange_pack": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
+    "sa_exchange_unpack": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "sa_get_status": (_I, [_P, _P]),
     "sa_last_error": (ctypes.c_char_p, [_P]),
     "sa_status_string": (ctypes.c_char_p, [_I]),
@@ -265,3 +270,17 @@ def sa_slot_of(cfg, chunk):
 
 def sa_get_status(handle, stream=0):
     return lib().sa_get_status(handle, _P(stream))
+
+
+def sa_exchange_block_bytes(B, T, C, D, G, split_dim, payload=SA_PAYLOAD_FP8):
+    """Bytes of one destination block of an exchange (0 if the shape is invalid)."""
+    return lib().sa_exchange_block_bytes(B, T, C, D, G, split_dim, payload)
+
+
+def sa_exchange_pack(x, B, T, C, D, G, split_dim, payload, buf, stream=0):
+    _check(lib().sa_exchange_pack(_P(x), B, T, C, D, G, split_dim, payload, _P(buf), _P(stream)))
+
+
+def sa_exchange_unpack(buf, B, T, C, D, G, split_dim, payload, y, stream=0):
+    _check(lib().sa_exchange_unpack(_P(buf), B, T, C, D, G, split_dim, payload, _P(y),
+                                    _P(stream)))

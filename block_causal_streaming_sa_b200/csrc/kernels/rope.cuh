@@ -66,10 +66,18 @@ __device__ __forceinline__ void st_v4(void* p, uint4 v) {
                : "memory");
 }
 
-// One block per token (b, l); thread t moves 16-byte chunk t % (D/8) of head
-// t / (D/8). blockIdx.y: 0 = K (bf16 in, rotated, fp16 out), 1 = V (bf16,
-// copied; rotated like K when second_is_key). Loads are fully coalesced (a token's H*D values are contiguous); each head's 2*D bytes are
-// stored contiguously into its [B, H, L_out, D] plane.
+// Tokens per block of rope_transpose_kernel: each thread issues the loads of all
+// of them before the first store, so enough bytes are in flight to cover HBM
+// latency (one token per thread leaves the copy latency-bound at about half the
+// bandwidth).
+constexpr int kRopeTokensPerBlock = 4;
+
+// Block x covers tokens (b, l) = kRopeTokensPerBlock * x .. + kRopeTokensPerBlock - 1
+// of the flattened [B * L] index; thread t moves 16-byte chunk t % (D/8) of head
+// t / (D/8) of each. blockIdx.y: 0 = K (bf16 in, rotated, fp16 out), 1 = V (bf16,
+// copied; rotated like K when second_is_key). Loads are fully coalesced (a
+// token's H*D values are contiguous); each head's 2*D bytes are stored
+// contiguously into its [B, H, L_out, D] plane.
 __global__ void rope_transpose_kernel(AppendParams p) {
   const int vec_per_head = p.D >> 3;
   const int t = threadIdx.x;
@@ -78,19 +86,28 @@ __global__ void rope_transpose_kernel(AppendParams p) {
   const __nv_bfloat16* in = is_v ? p.v_in : p.k_in;
   __nv_bfloat16* out = is_v ? p.v_out : p.k_out;
   if (in == nullptr) return;
-  const int tok = blockIdx.x;  // b * L + l
-  const int b = tok / p.L, l = tok - b * p.L;
   const int h = t / vec_per_head, c = t - h * vec_per_head;
-  const size_t src = (static_cast<size_t>(tok) * p.H + h) * p.D + c * 8;
-  const size_t dst = ((static_cast<size_t>(b) * p.H + h) * p.L_out + l) * p.D + c * 8;
-  uint4 v = ld_nc_v4(in + src);
-  if (!is_v || p.second_is_key) {
-    const int f = l / p.rope.frame_tokens;
-    const int y = (l / p.rope.tok_w) % p.rope.tok_h;
-    const int x = l % p.rope.tok_w;
-    v = rope_chunk(v, c, p.rope, f, y, x);
+  const int n_tok = p.B * p.L;
+  const int tok0 = blockIdx.x * kRopeTokensPerBlock;
+  uint4 v[kRopeTokensPerBlock];
+#pragma unroll
+  for (int k = 0; k < kRopeTokensPerBlock; ++k) {
+    const int tok = tok0 + k;
+    if (tok < n_tok) v[k] = ld_nc_v4(in + (static_cast<size_t>(tok) * p.H + h) * p.D + c * 8);
   }
-  st_v4(out + dst, v);
+#pragma unroll
+  for (int k = 0; k < kRopeTokensPerBlock; ++k) {
+    const int tok = tok0 + k;
+    if (tok >= n_tok) break;
+    const int b = tok / p.L, l = tok - b * p.L;
+    if (!is_v || p.second_is_key) {
+      const int f = l / p.rope.frame_tokens;
+      const int y = (l / p.rope.tok_w) % p.rope.tok_h;
+      const int x = l % p.rope.tok_w;
+      v[k] = rope_chunk(v[k], c, p.rope, f, y, x);
+    }
+    st_v4(out + ((static_cast<size_t>(b) * p.H + h) * p.L_out + l) * p.D + c * 8, v[k]);
+  }
 }
 
 }  // namespace sa

@@ -17,6 +17,7 @@
 #include "sa_internal.h"
 #include "kernels/attend_simt.cuh"
 #include "kernels/attend_tc.cuh"
+#include "kernels/exchange.cuh"
 #include "kernels/rope.cuh"
 
 using sa::AttendGroup;
@@ -344,7 +345,9 @@ int launch_rope_transpose(sa_handle* h, const void* K, const void* V, __nv_bfloa
   ap.second_is_key = second_is_key ? 1 : 0;
   ap.rope = h->rope();
   const int threads = static_cast<int>(align_up(static_cast<size_t>(d.H) * d.D / 8, 32));
-  dim3 grid(static_cast<unsigned>(d.B) * rows, V != nullptr ? 2 : 1);
+  const long long n_tok = 1LL * d.B * rows;
+  dim3 grid(static_cast<unsigned>((n_tok + sa::kRopeTokensPerBlock - 1) / sa::kRopeTokensPerBlock),
+            V != nullptr ? 2 : 1);
   sa::rope_transpose_kernel<<<grid, threads, 0, s>>>(ap);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
@@ -712,9 +715,98 @@ int append_chunk(sa_handle* h, int tier, const void* K, const void* V, int n_fra
   return SA_OK;
 }
 
+// ---------------------------------------------------------------- Ulysses exchange
+// Checks the sender's shape and fills the layout fields; false (and g_error) on a
+// bad argument.
+bool exchange_layout(int B, int T, int C, int D, int G, int split, int payload,
+                     sa::ExchangeParams* ep) {
+  if (B < 1 || T < 1 || C < 1 || G < 1 || (D != 64 && D != 128) || (split != 0 && split != 1) ||
+      (payload != SA_PAYLOAD_FP8 && payload != SA_PAYLOAD_BF16)) {
+    g_error = "exchange: need B, T, C, G >= 1, D in {64, 128}, split 0/1, a known payload";
+    return false;
+  }
+  if ((split == 0 ? T : C) % G != 0) {
+    g_error = "exchange: the split dimension must be a multiple of the rank count";
+    return false;
+  }
+  const long long n_vec = 1LL * B * T * C;
+  if (n_vec > (1LL << 32)) {
+    g_error = "exchange: tensor too large";
+    return false;
+  }
+  const long long per_block = n_vec / G;
+  std::memset(ep, 0, sizeof(*ep));
+  ep->B = B;
+  ep->T = T;
+  ep->C = C;
+  ep->D = D;
+  ep->G = G;
+  ep->split = split;
+  ep->fp8 = payload == SA_PAYLOAD_FP8 ? 1 : 0;
+  if (ep->fp8) {
+    ep->scale_off = static_cast<long long>(align_up(static_cast<size_t>(per_block) * D, 16));
+    ep->block_bytes =
+        ep->scale_off + static_cast<long long>(align_up(static_cast<size_t>(per_block) * 4, 16));
+  } else {
+    ep->block_bytes = per_block * D * 2;
+  }
+  return true;
+}
+
+int launch_exchange(bool pack, sa::ExchangeParams& ep, sa_stream stream) {
+  const long long n_vec = 1LL * ep.B * ep.T * ep.C;  // vectors of x (pack) and of y (unpack)
+  const unsigned grid = static_cast<unsigned>((n_vec + 7) / 8);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (pack)
+    ep.D == 128 ? sa::exchange_pack_kernel<128><<<grid, 256, 0, s>>>(ep)
+                : sa::exchange_pack_kernel<64><<<grid, 256, 0, s>>>(ep);
+  else
+    ep.D == 128 ? sa::exchange_unpack_kernel<128><<<grid, 256, 0, s>>>(ep)
+                : sa::exchange_unpack_kernel<64><<<grid, 256, 0, s>>>(ep);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    g_error = std::string("exchange launch: ") + cudaGetErrorString(e);
+    return SA_ERR_CUDA;
+  }
+  return SA_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+SA_API size_t sa_exchange_block_bytes(int B, int T, int C, int D, int G, int split_dim,
+                                      int payload) {
+  sa::ExchangeParams ep;
+  if (!exchange_layout(B, T, C, D, G, split_dim, payload, &ep)) return 0;
+  return static_cast<size_t>(ep.block_bytes);
+}
+
+SA_API int sa_exchange_pack(const void* x, int B, int T, int C, int D, int G, int split_dim,
+                            int payload, void* buf, sa_stream stream) {
+  sa::ExchangeParams ep;
+  if (!exchange_layout(B, T, C, D, G, split_dim, payload, &ep)) return SA_ERR_INVALID_ARG;
+  if (x == nullptr || buf == nullptr || !aligned16(x) || !aligned16(buf)) {
+    g_error = "exchange: x and buf must be non-NULL and 16-byte aligned";
+    return SA_ERR_INVALID_ARG;
+  }
+  ep.x = static_cast<const __nv_bfloat16*>(x);
+  ep.out = static_cast<uint8_t*>(buf);
+  return launch_exchange(true, ep, stream);
+}
+
+SA_API int sa_exchange_unpack(const void* buf, int B, int T, int C, int D, int G, int split_dim,
+                              int payload, void* y, sa_stream stream) {
+  sa::ExchangeParams ep;
+  if (!exchange_layout(B, T, C, D, G, split_dim, payload, &ep)) return SA_ERR_INVALID_ARG;
+  if (y == nullptr || buf == nullptr || !aligned16(y) || !aligned16(buf) || y == buf) {
+    g_error = "exchange: buf and y must be non-NULL, 16-byte aligned and distinct";
+    return SA_ERR_INVALID_ARG;
+  }
+  ep.in = static_cast<const uint8_t*>(buf);
+  ep.y = static_cast<__nv_bfloat16*>(y);
+  return launch_exchange(false, ep, stream);
+}
 
 SA_API int sa_validate_config(const sa_config* cfg) {
   std::string why;

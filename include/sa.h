@@ -297,6 +297,41 @@ SA_API int sa_plan(const sa_config* cfg, int32_t chunk, int32_t* ids, int32_t* s
 SA_API int sa_stream_plan(const sa_handle* h, int step_is_final, int n_frames, int32_t* ids,
                           int32_t* t_base, int32_t* lens, int cap);
 
+/* ---- Ulysses head sharding across GPUs ("Vidu S2：实时可交互、可编辑、可立体的视频生成",
+ * section 2.4; "Vidu S2 vs PixVerse R2", section 选择四：速度从哪里来: multi-GPU runs
+ * split load and activations with Ulysses context parallelism and quantise the
+ * tensors the GPUs exchange). G ranks each hold a contiguous 1/G of a chunk's
+ * tokens with all heads; an all-to-all gives each rank all tokens of H/G heads
+ * before attention, and a second one returns the output to token shards.
+ * These two calls are the local halves of such an exchange; the all-to-all of
+ * the G equal blocks between them is the caller's (NCCL over NVLink in the
+ * Python layer).
+ *
+ * x: [B, T, C, D] bf16 on the device (T tokens, C heads), 16-byte aligned.
+ * split_dim 1 (heads, before attention): block g holds heads g*C/G .. of every
+ * token; split_dim 0 (tokens, after attention): block g holds tokens g*T/G ..
+ * with every head. The split dimension must be a multiple of G.
+ * Payload SA_PAYLOAD_FP8: each (b, t, c) vector of D values is sent as fp8
+ * e4m3 codes (scale = max|x| / 448, code = e4m3(x / scale), nearest even,
+ * saturating; IEEE fp32 division) followed by its fp32 scale, D + 4 bytes
+ * instead of 2 D; on arrival code * scale (fp32) rounded to bf16. An all-zero
+ * vector has scale 0. SA_PAYLOAD_BF16 sends the values unchanged. Inputs must
+ * be finite.
+ * buf: G blocks of sa_exchange_block_bytes(...) bytes each, block g for rank g.
+ * sa_exchange_unpack takes the G blocks received (block s from rank s; every
+ * sender used the same B, T, C, D, G, split_dim, payload, which the call
+ * repeats) and writes y: split_dim 1 -> [B, G*T, C/G, D] (token shards in rank
+ * order); split_dim 0 -> [B, T/G, G*C, D] (head groups in rank order).
+ * Asynchronous on `stream`; SA_ERR_INVALID_ARG on a bad shape or pointer. */
+#define SA_PAYLOAD_FP8 0
+#define SA_PAYLOAD_BF16 1
+SA_API size_t sa_exchange_block_bytes(int B, int T, int C, int D, int G, int split_dim,
+                                      int payload); /* 0 if invalid; host only */
+SA_API int sa_exchange_pack(const void* x, int B, int T, int C, int D, int G, int split_dim,
+                            int payload, void* buf, sa_stream stream);
+SA_API int sa_exchange_unpack(const void* buf, int B, int T, int C, int D, int G, int split_dim,
+                              int payload, void* y, sa_stream stream);
+
 /* Slot of chunk id `chunk` in a tier (-1 if it is never stored). Host only. */
 SA_API int sa_slot_of(const sa_config* cfg, int32_t chunk);
 

@@ -160,3 +160,18 @@ def test_null_handle_new_calls_fail_cleanly():
         == sa.SA_ERR_INVALID_ARG
     assert lib.sa_stage_keys_frames(None, None, 1, None) == sa.SA_ERR_INVALID_ARG
     assert lib.sa_stream_plan(None, 0, 1, None, None, None, 16) < 0
+
+
+def test_exchange_block_bytes_and_shape_checks():
+    P8, P16 = sa.SA_PAYLOAD_FP8, sa.SA_PAYLOAD_BF16
+    # fp8: D code bytes per vector, then one fp32 scale per vector, each part 16-byte aligned
+    n = 1 * 2700 * 3  # vectors per block: B * T * H/G
+    assert sa.sa_exchange_block_bytes(1, 2700, 12, 128, 4, 1, P8) == n * 128 + n * 4
+    assert sa.sa_exchange_block_bytes(1, 10800, 3, 128, 4, 0, P16) == 2700 * 3 * 128 * 2
+    assert sa.sa_exchange_block_bytes(1, 3, 1, 64, 1, 0, P8) == 192 + 16  # 12 B of scales -> 16
+    for bad in [(1, 7, 3, 128, 2, 0, P8), (1, 8, 3, 128, 2, 1, P8), (1, 8, 4, 96, 2, 1, P8),
+                (0, 8, 4, 64, 2, 1, P8), (1, 8, 4, 64, 0, 1, P8), (1, 8, 4, 64, 2, 2, P8),
+                (1, 8, 4, 64, 2, 1, 7)]:
+        assert sa.sa_exchange_block_bytes(*bad) == 0, bad
+    with pytest.raises(sa.SaError):
+        sa.sa_exchange_pack(0, 1, 8, 4, 64, 2, 1, P8, 0)

@@ -74,3 +74,45 @@ def test_reference_arm_line_on_rank_zero():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def _a2a_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from block_causal_streaming_sa_b200.ulysses import all_to_all_blocks
+
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    nbytes = 24
+    # block g of rank r holds the byte pattern (r, g, i)
+    send = torch.tensor([(rank * 16 + g) * 3 + i % 3 for g in range(world) for i in range(nbytes)],
+                        dtype=torch.int64).to(torch.uint8)
+    recv = all_to_all_blocks(send)
+    dist.barrier()
+    dist.destroy_process_group()
+    out.put((rank, recv.tolist()))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_ulysses_block_all_to_all_on_gloo(world):
+    """The exchange primitive of the Ulysses layer: block s of rank r's result is
+    block r of rank s's send buffer (the layout sa_exchange_unpack expects)."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_a2a_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    nbytes = 24
+    for r in range(world):
+        want = [((s * 16 + r) * 3 + i % 3) % 256 for s in range(world) for i in range(nbytes)]
+        assert res[r] == want, r
