@@ -48,6 +48,8 @@ def parse_args():
                     help="block-sparse mode: share of 128x128 blocks skipped (seeded random mask)")
     ap.add_argument("--ulysses", action="store_true",
                     help="head-sharded attention over the ranks (Ulysses, fp8 exchange)")
+    ap.add_argument("--transport", choices=["nccl", "p2p"], default="nccl",
+                    help="Ulysses exchange: NCCL all-to-all, or quantise straight into peer memory")
     ap.add_argument("--editing", action="store_true",
                     help="frame-aligned editing attention (source frames of the chunk as extra keys)")
     ap.add_argument("--ref-frames", type=int, default=0,
@@ -333,7 +335,8 @@ def run_ours(args, w):
     if args.ulysses:
         from block_causal_streaming_sa_b200.ulysses import UlyssesAttention
 
-        layers = [UlyssesAttention(cfg, device=dev) for _ in range(w.layers)]
+        layers = [UlyssesAttention(cfg, device=dev, transport=args.transport)
+                  for _ in range(w.layers)]
     else:
         layers = [sa.StreamingAttention(cfg, device=dev) for _ in range(w.layers)]
     attn = layers[0]
@@ -533,7 +536,7 @@ def run_ours(args, w):
             "step": "all denoising attentions of one chunk (every layer) + noisy and clean appends",
             "l2": f"inputs larger than L2: {cache_bytes_read / 2**20:.0f} MiB of cached K/V "
                   f"read per attention vs {L2_BYTES / 2**20:.0f} MiB L2",
-            "parallelism": (f"ulysses{world}" if args.ulysses else
+            "parallelism": (f"ulysses{world}-{args.transport}" if args.ulysses else
                             f"replicas{world}" if world > 1 else "single"),
             "block_sparsity": args.sparsity,
             "ref_frames": args.ref_frames, "ref_tokens": ref_len,

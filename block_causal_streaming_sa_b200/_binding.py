@@ -26,6 +26,7 @@ SA_MAX_ATTENDED = 16
 SA_NOALLOC_MAX_KEY_BYTES = 64 << 20
 SA_PAYLOAD_FP8 = 0
 SA_PAYLOAD_BF16 = 1
+SA_IPC_HANDLE_BYTES = 64
 
 
 class SaConfig(ctypes.Structure):
@@ -85,6 +86,12 @@ _SIGNATURES = {
     "sa_exchange_block_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I]),
     "sa_exchange_pack": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "sa_exchange_unpack": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
+    "sa_exchange_pack_to": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_P), _P]),
+    "sa_ipc_alloc": (_I, [ctypes.c_size_t, ctypes.POINTER(_P)]),
+    "sa_ipc_free": (_I, [_P]),
+    "sa_ipc_handle": (_I, [_P, ctypes.c_char_p]),
+    "sa_ipc_open": (_I, [ctypes.c_char_p, ctypes.POINTER(_P)]),
+    "sa_ipc_close": (_I, [_P]),
     "sa_get_status": (_I, [_P, _P]),
     "sa_last_error": (ctypes.c_char_p, [_P]),
     "sa_status_string": (ctypes.c_char_p, [_I]),
@@ -284,3 +291,38 @@ def sa_exchange_pack(x, B, T, C, D, G, split_dim, payload, buf, stream=0):
 def sa_exchange_unpack(buf, B, T, C, D, G, split_dim, payload, y, stream=0):
     _check(lib().sa_exchange_unpack(_P(buf), B, T, C, D, G, split_dim, payload, _P(y),
                                     _P(stream)))
+
+
+def sa_exchange_pack_to(x, B, T, C, D, G, split_dim, payload, dst_blocks, stream=0):
+    """Pack with block g written straight to device address dst_blocks[g]."""
+    arr = (_P * G)(*[_P(int(a)) for a in dst_blocks])
+    _check(lib().sa_exchange_pack_to(_P(x), B, T, C, D, G, split_dim, payload, arr, _P(stream)))
+
+
+def sa_ipc_handle(dev_ptr):
+    """The CUDA IPC handle (bytes) of the allocation starting at dev_ptr."""
+    buf = ctypes.create_string_buffer(SA_IPC_HANDLE_BYTES)
+    _check(lib().sa_ipc_handle(_P(dev_ptr), buf))
+    return buf.raw
+
+
+def sa_ipc_open(handle):
+    """Map another process's allocation; returns its device address here."""
+    out = _P()
+    _check(lib().sa_ipc_open(bytes(handle), ctypes.byref(out)))
+    return out.value
+
+
+def sa_ipc_close(dev_ptr):
+    _check(lib().sa_ipc_close(_P(dev_ptr)))
+
+
+def sa_ipc_alloc(nbytes):
+    """A whole device allocation that can be shared by CUDA IPC; returns its address."""
+    out = _P()
+    _check(lib().sa_ipc_alloc(nbytes, ctypes.byref(out)))
+    return out.value
+
+
+def sa_ipc_free(dev_ptr):
+    _check(lib().sa_ipc_free(_P(dev_ptr)))

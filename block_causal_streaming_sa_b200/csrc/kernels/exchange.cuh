@@ -8,6 +8,9 @@
 // g holds tokens g*T/G .. with every head. Inside a block the vectors are in
 // [B][T'][C'] order. fp8 payload: codes [B][T'][C'][D] e4m3, then, 16-byte
 // aligned, one fp32 scale per vector; bf16 payload: the values as they are.
+// With dst[], pack writes block g straight to dst[g]: for a peer's receive buffer
+// mapped into this process (CUDA IPC over NVLink) the quantisation and the
+// transfer are one pass, with no staging copy and no separate collective.
 // unpack: the G blocks received (block s from rank s, each laid out as the
 // sender's pack made it) -> y: split 1: [B][G*T'][C'][D] (token shards in rank
 // order); split 0: [B][T'][G*C'][D] (head groups in rank order).
@@ -26,10 +29,14 @@
 
 namespace sa {
 
+constexpr int kMaxExchangeRanks = 64;
+
 struct ExchangeParams {
   const __nv_bfloat16* x;  // pack input
   const uint8_t* in;       // unpack input (G blocks)
-  uint8_t* out;            // pack output (G blocks)
+  uint8_t* out;            // pack output (G blocks), or null with dst[]
+  uint8_t* dst[kMaxExchangeRanks];  // pack output: where block g goes (e.g. a peer's
+                                    // receive buffer mapped into this process)
   __nv_bfloat16* y;        // unpack output
   int B, T, C, D, G;       // the sender's x shape and the rank count
   int split;               // 0: tokens, 1: heads
@@ -85,7 +92,7 @@ __global__ void __launch_bounds__(256) exchange_pack_kernel(ExchangeParams p) {
   int g;
   long long v;
   exchange_place(p, b, t, c, g, v);
-  uint8_t* blk = p.out + g * p.block_bytes;
+  uint8_t* blk = p.out != nullptr ? p.out + g * p.block_bytes : p.dst[g];
   const __nv_bfloat16* src = p.x + vec * D + lane * E;
   // E bf16 values of this lane as E / 2 packed 32-bit words
   uint32_t w[E / 2];
@@ -101,6 +108,7 @@ __global__ void __launch_bounds__(256) exchange_pack_kernel(ExchangeParams p) {
                                                 lane * E);
 #pragma unroll
     for (int i = 0; i < E / 2; ++i) dst[i] = w[i];
+    if (p.out == nullptr) __threadfence_system();  // peer stores performed before the kernel ends
     return;
   }
   float f[E];
@@ -127,6 +135,7 @@ __global__ void __launch_bounds__(256) exchange_pack_kernel(ExchangeParams p) {
   else
     *reinterpret_cast<uint16_t*>(codes) = q[0];
   if (lane == 0) reinterpret_cast<float*>(blk + p.scale_off)[v] = scale;
+  if (p.out == nullptr) __threadfence_system();  // peer stores performed before the kernel ends
 }
 
 // One warp per vector of y.

@@ -795,6 +795,96 @@ SA_API int sa_exchange_pack(const void* x, int B, int T, int C, int D, int G, in
   return launch_exchange(true, ep, stream);
 }
 
+SA_API int sa_exchange_pack_to(const void* x, int B, int T, int C, int D, int G, int split_dim,
+                               int payload, void* const* dst_blocks, sa_stream stream) {
+  sa::ExchangeParams ep;
+  if (!exchange_layout(B, T, C, D, G, split_dim, payload, &ep)) return SA_ERR_INVALID_ARG;
+  if (G > sa::kMaxExchangeRanks) {
+    g_error = "exchange: more ranks than sa_exchange_pack_to supports (64)";
+    return SA_ERR_UNSUPPORTED;
+  }
+  if (x == nullptr || dst_blocks == nullptr || !aligned16(x)) {
+    g_error = "exchange: x and dst_blocks must be non-NULL, x 16-byte aligned";
+    return SA_ERR_INVALID_ARG;
+  }
+  for (int g = 0; g < G; ++g) {
+    if (dst_blocks[g] == nullptr || !aligned16(dst_blocks[g])) {
+      g_error = "exchange: every destination block must be non-NULL and 16-byte aligned";
+      return SA_ERR_INVALID_ARG;
+    }
+    ep.dst[g] = static_cast<uint8_t*>(dst_blocks[g]);
+  }
+  ep.x = static_cast<const __nv_bfloat16*>(x);
+  ep.out = nullptr;
+  return launch_exchange(true, ep, stream);
+}
+
+SA_API int sa_ipc_alloc(size_t bytes, void** dev_ptr_out) {
+  if (dev_ptr_out == nullptr || bytes == 0) {
+    g_error = "ipc: NULL output or zero size";
+    return SA_ERR_INVALID_ARG;
+  }
+  *dev_ptr_out = nullptr;
+  cudaError_t e = cudaMalloc(dev_ptr_out, bytes);
+  if (e != cudaSuccess) {
+    g_error = std::string("cudaMalloc of an IPC buffer: ") + cudaGetErrorString(e);
+    return SA_ERR_CUDA;
+  }
+  return SA_OK;
+}
+
+SA_API int sa_ipc_free(void* dev_ptr) {
+  if (dev_ptr == nullptr) return SA_OK;
+  cudaError_t e = cudaFree(dev_ptr);
+  if (e != cudaSuccess) {
+    g_error = std::string("cudaFree of an IPC buffer: ") + cudaGetErrorString(e);
+    return SA_ERR_CUDA;
+  }
+  return SA_OK;
+}
+
+SA_API int sa_ipc_handle(const void* dev_ptr, void* handle_out) {
+  if (dev_ptr == nullptr || handle_out == nullptr) {
+    g_error = "ipc: NULL argument";
+    return SA_ERR_INVALID_ARG;
+  }
+  cudaIpcMemHandle_t hdl;
+  cudaError_t e = cudaIpcGetMemHandle(&hdl, const_cast<void*>(dev_ptr));
+  if (e != cudaSuccess) {
+    g_error = std::string("cudaIpcGetMemHandle: ") + cudaGetErrorString(e);
+    return SA_ERR_CUDA;
+  }
+  static_assert(sizeof(hdl) == SA_IPC_HANDLE_BYTES, "IPC handle size");
+  std::memcpy(handle_out, &hdl, sizeof(hdl));
+  return SA_OK;
+}
+
+SA_API int sa_ipc_open(const void* handle, void** dev_ptr_out) {
+  if (handle == nullptr || dev_ptr_out == nullptr) {
+    g_error = "ipc: NULL argument";
+    return SA_ERR_INVALID_ARG;
+  }
+  cudaIpcMemHandle_t hdl;
+  std::memcpy(&hdl, handle, sizeof(hdl));
+  *dev_ptr_out = nullptr;
+  cudaError_t e = cudaIpcOpenMemHandle(dev_ptr_out, hdl, cudaIpcMemLazyEnablePeerAccess);
+  if (e != cudaSuccess) {
+    g_error = std::string("cudaIpcOpenMemHandle: ") + cudaGetErrorString(e);
+    return SA_ERR_CUDA;
+  }
+  return SA_OK;
+}
+
+SA_API int sa_ipc_close(void* dev_ptr) {
+  if (dev_ptr == nullptr) return SA_OK;
+  cudaError_t e = cudaIpcCloseMemHandle(dev_ptr);
+  if (e != cudaSuccess) {
+    g_error = std::string("cudaIpcCloseMemHandle: ") + cudaGetErrorString(e);
+    return SA_ERR_CUDA;
+  }
+  return SA_OK;
+}
+
 SA_API int sa_exchange_unpack(const void* buf, int B, int T, int C, int D, int G, int split_dim,
                               int payload, void* y, sa_stream stream) {
   sa::ExchangeParams ep;

@@ -332,6 +332,31 @@ SA_API int sa_exchange_pack(const void* x, int B, int T, int C, int D, int G, in
 SA_API int sa_exchange_unpack(const void* buf, int B, int T, int C, int D, int G, int split_dim,
                               int payload, void* y, sa_stream stream);
 
+/* sa_exchange_pack that writes block g straight to dst_blocks[g] (a host array
+ * of G device pointers, each 16-byte aligned, e.g. this rank's slot in rank g's
+ * receive buffer mapped with sa_ipc_open): quantisation and transfer in one
+ * pass over peer memory, no staging copy, no separate collective. The caller
+ * orders the receivers' sa_exchange_unpack after every sender's launch (a
+ * barrier) and keeps a receiver from reusing a buffer that a sender may still
+ * be writing (two receive buffers used in turn). G <= 64. */
+SA_API int sa_exchange_pack_to(const void* x, int B, int T, int C, int D, int G, int split_dim,
+                               int payload, void* const* dst_blocks, sa_stream stream);
+
+/* CUDA IPC of device buffers between processes (the peer mappings of
+ * sa_exchange_pack_to): sa_ipc_alloc / sa_ipc_free make and release a whole
+ * cudaMalloc allocation on the current device (a receive buffer; the only
+ * allocations this library makes itself); sa_ipc_handle writes the
+ * SA_IPC_HANDLE_BYTES-byte handle of such an allocation (dev_ptr = its start);
+ * sa_ipc_open maps another process's handle into this one (peer access enabled
+ * on first use); sa_ipc_close unmaps it. A handle cannot be opened in the
+ * process that made it. */
+#define SA_IPC_HANDLE_BYTES 64
+SA_API int sa_ipc_alloc(size_t bytes, void** dev_ptr_out);
+SA_API int sa_ipc_free(void* dev_ptr);
+SA_API int sa_ipc_handle(const void* dev_ptr, void* handle_out);
+SA_API int sa_ipc_open(const void* handle, void** dev_ptr_out);
+SA_API int sa_ipc_close(void* dev_ptr);
+
 /* Slot of chunk id `chunk` in a tier (-1 if it is never stored). Host only. */
 SA_API int sa_slot_of(const sa_config* cfg, int32_t chunk);
 
