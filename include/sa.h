@@ -31,6 +31,10 @@
  *    passed as sa_stream; NULL is the legacy default stream). After sa_create,
  *    sa_append_chunk / sa_stage_keys / sa_attend_staged / sa_attend allocate no
  *    memory and never synchronise the host.
+ *  - The device calls can be captured into a CUDA graph. A captured attention
+ *    keeps the plan of the chunk it was captured for (attended chunks, slots
+ *    and relocated positions are launch arguments): replay it for that chunk's
+ *    steps of the same tier, with new contents in the same input buffers.
  *  - Every call returns an sa_status. On error nothing is launched and the
  *    handle's counters are unchanged; sa_last_error() explains the failure.
  *  - A handle is not thread-safe: one host thread drives one handle.
