@@ -78,7 +78,7 @@ def kernel_traffic(kernel_file, workload):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the kernel source as it is now; else None."""
     src = os.path.join(ROOT, "block_causal_streaming_sa_b200", "csrc", "kernels", kernel_file)
-    summ = os.path.join(ROOT, "profiles", f"attend_tc_{workload}.md")
+    summ = os.path.join(ROOT, "profiles", f"attend_tc_{workload}.txt")
     try:
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
         text = open(summ).read()

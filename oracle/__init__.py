@@ -29,7 +29,8 @@ Sources (web pages, cited by title and section):
             causal mask; sliding-window context plus a rolling KV cache keep
             memory bounded.
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent (the prefix, variable-length, editing and
+exchange readings R13-R16 are stated in stream.py, editing.py and exchange.py):
   R1  the window W counts the current chunk: keys = (S + W) * L.
   R2  inside a chunk attention is bidirectional.
   R3  relocated temporal position of frame f of chunk j is rank(j) * F + f,

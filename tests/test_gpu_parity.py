@@ -145,7 +145,7 @@ FULL = [
 
 @pytest.mark.parametrize("case", FULL, ids=[c[0] for c in FULL])
 def test_full_size_sampled_rows(case):
-    """BASELINE-sized configs in the bench's launch configuration: the first
+    """The full-size workloads in the bench's launch configuration: the first
     chunk (no cache) and, after eviction has begun, one noisy and one clean
     step, on >= 256 sampled query rows per checked (b, h)."""
     name, heads, batches, nrows = case
