@@ -478,45 +478,103 @@ __global__ void __launch_bounds__(384, 1)
             ok = ptx::mbar_wait(bar(T::QREADY(i)), rr & 1, abort_flag, p.status);
           continue;
         }
-        int sk = 0, sv = 0;
-        if (!take_stage(sk)) break;
-        ptx::tc_fence_after();
-        for (int i = 0; i < 2; ++i) {
-          if (!ptx::mbar_wait(bar(T::QREADY(i)), rr & 1, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          ptx::tc_fence_after();
-          issue_s(i, sk);
-          ptx::umma_commit(bar(T::SFULL(i)));
-        }
-        if (!ok) break;
-        ptx::umma_commit(bar(T::EMPTY(sk)));
-        for (bool first = true; ok && u < hi; first = false) {
-          const int nu = next_visited(mo, mo1, u + 1, hi);
-          const bool has_next = nu < hi;
-          if (!take_stage(sv) || (has_next && !take_stage(sk))) {
-            ok = false;
-            break;
-          }
+        if constexpr (!kSparse) {
+          int sk = 0, sv = 0;
+          if (!take_stage(sk)) break;
           ptx::tc_fence_after();
           for (int i = 0; i < 2; ++i) {
-            if (!ptx::mbar_wait(bar(T::PFULL(i)), pf_phase[i], abort_flag, p.status)) {
+            if (!ptx::mbar_wait(bar(T::QREADY(i)), rr & 1, abort_flag, p.status)) {
               ok = false;
               break;
             }
-            pf_phase[i] ^= 1u;
             ptx::tc_fence_after();
-            issue_pv(i, sv, !first);
-            if (i == 1) ptx::umma_commit(bar(T::EMPTY(sv)));
-            if (!has_next) ptx::umma_commit(bar(T::OFINAL(i)));
-            if (has_next) {
+            issue_s(i, sk);
+            ptx::umma_commit(bar(T::SFULL(i)));
+          }
+          if (!ok) break;
+          ptx::umma_commit(bar(T::EMPTY(sk)));
+          for (bool first = true; ok && u < hi; first = false) {
+            const int nu = next_visited(mo, mo1, u + 1, hi);
+            const bool has_next = nu < hi;
+            if (!take_stage(sv) || (has_next && !take_stage(sk))) {
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
+            for (int i = 0; i < 2; ++i) {
+              if (!ptx::mbar_wait(bar(T::PFULL(i)), pf_phase[i], abort_flag, p.status)) {
+                ok = false;
+                break;
+              }
+              pf_phase[i] ^= 1u;
+              ptx::tc_fence_after();
+              issue_pv(i, sv, !first);
+              if (i == 1) ptx::umma_commit(bar(T::EMPTY(sv)));
+              if (!has_next) ptx::umma_commit(bar(T::OFINAL(i)));
+              if (has_next) {
+                issue_s(i, sk);
+                ptx::umma_commit(bar(T::SFULL(i)));
+              }
+            }
+            if (ok && has_next) ptx::umma_commit(bar(T::EMPTY(sk)));
+            u = nu;
+          }
+        } else {
+          // Block-sparse: query tile i takes part in key tile t when its block is
+          // flagged (S, softmax and P.V for that tile only); the key stream is the
+          // union of both tiles' blocks.
+          auto wants = [&](int i, int t) { return flag(i == 0 ? mo : mo1, t); };
+          int sk = 0, sv = 0;
+          if (!take_stage(sk)) break;
+          ptx::tc_fence_after();
+          for (int i = 0; i < 2; ++i) {
+            if (!ptx::mbar_wait(bar(T::QREADY(i)), rr & 1, abort_flag, p.status)) {
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
+            if (wants(i, u)) {
               issue_s(i, sk);
               ptx::umma_commit(bar(T::SFULL(i)));
             }
           }
-          if (ok && has_next) ptx::umma_commit(bar(T::EMPTY(sk)));
-          u = nu;
+          if (!ok) break;
+          ptx::umma_commit(bar(T::EMPTY(sk)));
+          bool issued[2] = {false, false};  // a P.V of tile i issued in this unit
+          while (ok && u < hi) {
+            const int nu = next_visited(mo, mo1, u + 1, hi);
+            const bool has_next = nu < hi;
+            if (!take_stage(sv) || (has_next && !take_stage(sk))) {
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
+            for (int i = 0; i < 2; ++i) {
+              if (wants(i, u)) {
+                if (!ptx::mbar_wait(bar(T::PFULL(i)), pf_phase[i], abort_flag, p.status)) {
+                  ok = false;
+                  break;
+                }
+                pf_phase[i] ^= 1u;
+                ptx::tc_fence_after();
+                issue_pv(i, sv, issued[i]);
+                issued[i] = true;
+              }
+              if (i == 1) ptx::umma_commit(bar(T::EMPTY(sv)));  // V read by both P.V
+              // S of tile i's next key tile; its S region is free: the softmax has
+              // published P of its previous tile, whose P.V is issued before this.
+              if (has_next && wants(i, nu)) {
+                issue_s(i, sk);
+                ptx::umma_commit(bar(T::SFULL(i)));
+              }
+            }
+            if (!ok) break;
+            if (has_next) ptx::umma_commit(bar(T::EMPTY(sk)));
+            u = nu;
+          }
+          if (ok)  // O of a query tile with at least one block is final
+            for (int i = 0; i < 2; ++i)
+              if (issued[i]) ptx::umma_commit(bar(T::OFINAL(i)));
         }
       }
       // Every MMA issued so far must finish before TMEM is released.
@@ -556,12 +614,13 @@ __global__ void __launch_bounds__(384, 1)
         mask_rows(w, mo, mo1);
         own = i == 0 ? mo : mo1;
       }
-      // First chunk with a visited key tile (the query tile is rotated for it).
-      // Frame-aligned units visit every group, the last one partly.
+      // First chunk with a key tile of this query tile (it is rotated for it).
+      // Sparse: the tiles flagged for this query tile only; frame-aligned units
+      // visit every group, the last one partly.
       int g0 = glo;
       bool any_tile = true;
       if (kSparse) {
-        const int u0 = next_visited(mo, mo1, gstart[glo], gstart[ghi]);
+        const int u0 = next_visited(own, -1, gstart[glo], gstart[ghi]);
         any_tile = u0 < gstart[ghi];
         while (g0 + 1 < ghi && u0 >= gstart[g0 + 1]) ++g0;
       }
@@ -592,15 +651,14 @@ __global__ void __launch_bounds__(384, 1)
           t1 = mo1 - gstart[g];
         }
         for (int t = t0; t < t1; ++t) {
-          if (kSparse && next_visited(mo, mo1, gstart[g] + t, gstart[g] + t + 1) != gstart[g] + t)
-            continue;
+          if (kSparse && !flag(own, gstart[g] + t)) continue;
           if (!ptx::mbar_wait(bar(T::SFULL(i)), s_phase, abort_flag, p.status)) {
             ok = false;
             break;
           }
           s_phase ^= 1u;
           ptx::tc_fence_after();
-          if (!kSparse || flag(own, gstart[g] + t)) {
+          {
             // The whole score row (128 fp32) in one round trip; keys past the chunk end
             // masked, and in a source tile every key outside the row's own frame.
             int c_lo = 0, c_hi = min(T::BN, len - t * T::BN);
@@ -686,19 +744,12 @@ __global__ void __launch_bounds__(384, 1)
                 ptx::tmem_st32(tO + j * 32, o);
               }
             }
-          } else {
-            // Block flagged for the partner query tile only: P = 0 here.
-            uint32_t zero[16];
-#pragma unroll
-            for (int c = 0; c < 16; ++c) zero[c] = 0u;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) ptx::tmem_st16(tS + 64 + j * 16, zero);
           }
           // Chunk switch: the next key tile lies in a later chunk; turn the query
           // tile's temporal band to that chunk's relocated offset first.
           int gn = g;
           if (kSparse) {
-            const int nu = next_visited(mo, mo1, gstart[g] + t + 1, gstart[ghi]);
+            const int nu = next_visited(own, -1, gstart[g] + t + 1, gstart[ghi]);
             if (nu < gstart[ghi] && nu >= gstart[g + 1])
               while (gn + 1 < ghi && nu >= gstart[gn + 1]) ++gn;
           } else if (t == t1 - 1 && g + 1 < ghi) {
