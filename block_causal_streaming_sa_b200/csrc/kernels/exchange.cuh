@@ -79,113 +79,139 @@ __device__ __forceinline__ float2 e4m3x2_to_f32(uint16_t v) {
   return f;
 }
 
-// One warp per vector of x; lane l holds elements l*E .. l*E + E - 1 (E = D / 32).
+// Vectors per warp: each lane issues the loads of all of them before the first
+// store, so enough bytes are in flight to cover memory latency.
+constexpr int kExchangeVecPerWarp = 4;
+
+// One warp per kExchangeVecPerWarp consecutive vectors of x; lane l holds
+// elements l*E .. l*E + E - 1 of each (E = D / 32).
 template <int D>
 __global__ void __launch_bounds__(256) exchange_pack_kernel(ExchangeParams p) {
-  constexpr int E = D / 32;
-  const long long vec = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  constexpr int E = D / 32, V = kExchangeVecPerWarp;
+  const long long vec0 = (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * V;
   const int lane = threadIdx.x & 31;
-  if (vec >= static_cast<long long>(p.B) * p.T * p.C) return;
-  const int c = static_cast<int>(vec % p.C);
-  const long long bt = vec / p.C;
-  const int t = static_cast<int>(bt % p.T), b = static_cast<int>(bt / p.T);
-  int g;
-  long long v;
-  exchange_place(p, b, t, c, g, v);
-  uint8_t* blk = p.out != nullptr ? p.out + g * p.block_bytes : p.dst[g];
-  const __nv_bfloat16* src = p.x + vec * D + lane * E;
-  // E bf16 values of this lane as E / 2 packed 32-bit words
-  uint32_t w[E / 2];
-  if constexpr (E == 4) {
-    const uint2 u = *reinterpret_cast<const uint2*>(src);
-    w[0] = u.x;
-    w[1] = u.y;
-  } else {
-    w[0] = *reinterpret_cast<const uint32_t*>(src);
+  const long long n_vec = static_cast<long long>(p.B) * p.T * p.C;
+  // E bf16 values of this lane as E / 2 packed 32-bit words, for each vector
+  uint32_t w[V][E / 2];
+#pragma unroll
+  for (int k = 0; k < V; ++k) {
+    if (vec0 + k >= n_vec) break;
+    const __nv_bfloat16* src = p.x + (vec0 + k) * D + lane * E;
+    if constexpr (E == 4) {
+      const uint2 u = *reinterpret_cast<const uint2*>(src);
+      w[k][0] = u.x;
+      w[k][1] = u.y;
+    } else {
+      w[k][0] = *reinterpret_cast<const uint32_t*>(src);
+    }
   }
-  if (!p.fp8) {
-    uint32_t* dst = reinterpret_cast<uint32_t*>(reinterpret_cast<__nv_bfloat16*>(blk) + v * D +
-                                                lane * E);
 #pragma unroll
-    for (int i = 0; i < E / 2; ++i) dst[i] = w[i];
-    if (p.out == nullptr) __threadfence_system();  // peer stores performed before the kernel ends
-    return;
+  for (int k = 0; k < V; ++k) {
+    const long long vec = vec0 + k;
+    if (vec >= n_vec) break;
+    const int c = static_cast<int>(vec % p.C);
+    const long long bt = vec / p.C;
+    const int t = static_cast<int>(bt % p.T), b = static_cast<int>(bt / p.T);
+    int g;
+    long long v;
+    exchange_place(p, b, t, c, g, v);
+    uint8_t* blk = p.out != nullptr ? p.out + g * p.block_bytes : p.dst[g];
+    if (!p.fp8) {
+      uint32_t* dst = reinterpret_cast<uint32_t*>(reinterpret_cast<__nv_bfloat16*>(blk) + v * D +
+                                                  lane * E);
+#pragma unroll
+      for (int i = 0; i < E / 2; ++i) dst[i] = w[k][i];
+      continue;
+    }
+    float f[E];
+#pragma unroll
+    for (int i = 0; i < E / 2; ++i) {
+      f[2 * i] = __uint_as_float(w[k][i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[k][i] & 0xFFFF0000u);
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < E; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const float scale = __fdiv_rn(amax, kE4m3Max);
+    uint8_t* codes = blk + v * D + lane * E;
+    uint16_t q[E / 2];
+#pragma unroll
+    for (int i = 0; i < E / 2; ++i)
+      q[i] = scale > 0.f ? e4m3x2(__fdiv_rn(f[2 * i], scale), __fdiv_rn(f[2 * i + 1], scale))
+                         : static_cast<uint16_t>(0);
+    if constexpr (E == 4)
+      *reinterpret_cast<uint32_t*>(codes) = static_cast<uint32_t>(q[0]) |
+                                            (static_cast<uint32_t>(q[E / 2 - 1]) << 16);
+    else
+      *reinterpret_cast<uint16_t*>(codes) = q[0];
+    if (lane == 0) reinterpret_cast<float*>(blk + p.scale_off)[v] = scale;
   }
-  float f[E];
-#pragma unroll
-  for (int i = 0; i < E / 2; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < E; ++i) amax = fmaxf(amax, fabsf(f[i]));
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  const float scale = __fdiv_rn(amax, kE4m3Max);
-  uint8_t* codes = blk + v * D + lane * E;
-  uint16_t q[E / 2];
-#pragma unroll
-  for (int i = 0; i < E / 2; ++i)
-    q[i] = scale > 0.f ? e4m3x2(__fdiv_rn(f[2 * i], scale), __fdiv_rn(f[2 * i + 1], scale))
-                       : static_cast<uint16_t>(0);
-  if constexpr (E == 4)
-    *reinterpret_cast<uint32_t*>(codes) = static_cast<uint32_t>(q[0]) |
-                                          (static_cast<uint32_t>(q[E / 2 - 1]) << 16);
-  else
-    *reinterpret_cast<uint16_t*>(codes) = q[0];
-  if (lane == 0) reinterpret_cast<float*>(blk + p.scale_off)[v] = scale;
   if (p.out == nullptr) __threadfence_system();  // peer stores performed before the kernel ends
 }
 
-// One warp per vector of y.
+// One warp per kExchangeVecPerWarp consecutive vectors of y.
 template <int D>
 __global__ void __launch_bounds__(256) exchange_unpack_kernel(ExchangeParams p) {
-  constexpr int E = D / 32;
+  constexpr int E = D / 32, V = kExchangeVecPerWarp;
   const int Tb = p.split == 0 ? p.T / p.G : p.T;
   const int Cb = p.split == 1 ? p.C / p.G : p.C;
   // y is [B][Ty][Cy][D]
   const int Ty = p.split == 1 ? p.G * Tb : Tb;
   const int Cy = p.split == 0 ? p.G * Cb : Cb;
-  const long long vec = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const long long vec0 = (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * V;
   const int lane = threadIdx.x & 31;
-  if (vec >= static_cast<long long>(p.B) * Ty * Cy) return;
-  const int cy = static_cast<int>(vec % Cy);
-  const long long bt = vec / Cy;
-  const int ty = static_cast<int>(bt % Ty), b = static_cast<int>(bt / Ty);
-  int s, tl = ty, cl = cy;
-  if (p.split == 1) {
-    s = ty / Tb;
-    tl = ty - s * Tb;
-  } else {
-    s = cy / Cb;
-    cl = cy - s * Cb;
-  }
-  const long long v = (static_cast<long long>(b) * Tb + tl) * Cb + cl;
-  const uint8_t* blk = p.in + s * p.block_bytes;
-  __nv_bfloat16* dst = p.y + vec * D + lane * E;
-  uint32_t* out = reinterpret_cast<uint32_t*>(dst);
-  if (!p.fp8) {
-    const uint32_t* src = reinterpret_cast<const uint32_t*>(
-        reinterpret_cast<const __nv_bfloat16*>(blk) + v * D + lane * E);
+  const long long n_vec = static_cast<long long>(p.B) * Ty * Cy;
+  uint32_t raw[V][E / 2];  // bf16 words, or the E code bytes in raw[k][0] (fp8)
+  float scale[V];
 #pragma unroll
-    for (int i = 0; i < E / 2; ++i) out[i] = src[i];
-    return;
-  }
-  const float scale = reinterpret_cast<const float*>(blk + p.scale_off)[v];
-  const uint8_t* codes = blk + v * D + lane * E;
-  uint16_t q[E / 2];
-  if constexpr (E == 4) {
-    const uint32_t u = *reinterpret_cast<const uint32_t*>(codes);
-    q[0] = static_cast<uint16_t>(u);
-    q[E / 2 - 1] = static_cast<uint16_t>(u >> 16);
-  } else {
-    q[0] = *reinterpret_cast<const uint16_t*>(codes);
+  for (int k = 0; k < V; ++k) {
+    const long long vec = vec0 + k;
+    if (vec >= n_vec) break;
+    const int cy = static_cast<int>(vec % Cy);
+    const long long bt = vec / Cy;
+    const int ty = static_cast<int>(bt % Ty), b = static_cast<int>(bt / Ty);
+    int s, tl = ty, cl = cy;
+    if (p.split == 1) {
+      s = ty / Tb;
+      tl = ty - s * Tb;
+    } else {
+      s = cy / Cb;
+      cl = cy - s * Cb;
+    }
+    const long long v = (static_cast<long long>(b) * Tb + tl) * Cb + cl;
+    const uint8_t* blk = p.in + s * p.block_bytes;
+    if (!p.fp8) {
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(
+          reinterpret_cast<const __nv_bfloat16*>(blk) + v * D + lane * E);
+#pragma unroll
+      for (int i = 0; i < E / 2; ++i) raw[k][i] = src[i];
+    } else {
+      scale[k] = reinterpret_cast<const float*>(blk + p.scale_off)[v];
+      const uint8_t* codes = blk + v * D + lane * E;
+      if constexpr (E == 4)
+        raw[k][0] = *reinterpret_cast<const uint32_t*>(codes);
+      else
+        raw[k][0] = *reinterpret_cast<const uint16_t*>(codes);
+    }
   }
 #pragma unroll
-  for (int i = 0; i < E / 2; ++i) {
-    const float2 fv = e4m3x2_to_f32(q[i]);
-    out[i] = ptx::pack_bf16x2(__fmul_rn(fv.x, scale), __fmul_rn(fv.y, scale));
+  for (int k = 0; k < V; ++k) {
+    const long long vec = vec0 + k;
+    if (vec >= n_vec) break;
+    uint32_t* out = reinterpret_cast<uint32_t*>(p.y + vec * D + lane * E);
+    if (!p.fp8) {
+#pragma unroll
+      for (int i = 0; i < E / 2; ++i) out[i] = raw[k][i];
+      continue;
+    }
+#pragma unroll
+    for (int i = 0; i < E / 2; ++i) {
+      const float2 fv = e4m3x2_to_f32(static_cast<uint16_t>(raw[k][0] >> (16 * i)));
+      out[i] = ptx::pack_bf16x2(__fmul_rn(fv.x, scale[k]), __fmul_rn(fv.y, scale[k]));
+    }
   }
 }
 
