@@ -101,6 +101,18 @@ def normal_bf16(seed, shape, scale=1.0, outlier_frac=0.0, outlier_mag=8.0):
     return torch.from_numpy(out.reshape(shape)).to(torch.bfloat16)
 
 
+def device_normal_bf16(seed, shape, device):
+    """N(0, 1) bf16 tensor made on `device` by torch's seeded generator of that
+    device, for inputs too large to draw on the host (tens of GB). Deterministic
+    for a given seed, shape and device type; slices of it are copied to the host
+    where a check needs them."""
+    import torch
+
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed) & 0x7FFFFFFFFFFFFFFF)
+    return torch.randn(shape, generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+
 @dataclass(frozen=True)
 class Workload:
     """Shape of one synthetic workload (all tensors [B, L, H, D] bf16)."""
