@@ -221,6 +221,25 @@ def cpu_baseline(w, seconds):
                       f"{dt:.1f} s of float64 numpy on the host"}
 
 
+def workload_config(w, args, world):
+    """The `config` object of a bench line (both arms describe the same workload)."""
+    cache_bytes_read = 2 * (w.kv_len - w.chunk_len) * w.batch * w.heads * w.head_dim * 2
+    return {
+        "workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
+        "chunk_tokens": w.chunk_len, "kv_tokens": w.kv_len, "sink_chunks": w.sink,
+        "window_chunks": w.window, "denoise_steps_per_chunk": w.steps, "layers": w.layers,
+        "step": "all denoising attentions of one chunk (every layer) + noisy and clean appends",
+        "l2": f"inputs larger than L2: {cache_bytes_read / 2**20:.0f} MiB of cached K/V "
+              f"read per attention vs {L2_BYTES / 2**20:.0f} MiB L2",
+        "parallelism": (f"ulysses{world}-{args.transport}" if args.ulysses else
+                        f"replicas{world}" if world > 1 else "single"),
+        "block_sparsity": args.sparsity,
+        "ref_frames": args.ref_frames,
+        "ref_tokens": args.ref_frames * w.tok_h * w.tok_w,
+        "frame_aligned_editing": args.editing,
+    }
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -241,7 +260,7 @@ def run_reference(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
-        "config": {"workload": w.name, "sample": sample},
+        "config": dict(workload_config(w, args, args.gpus), sample=sample),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -542,7 +561,6 @@ def run_ours(args, w):
     append_bytes = appends_per_chunk * 2 * 2 * (w.batch * w.chunk_len * w.heads * w.head_dim * 2)
     # (per append of one tier: K and V, each read once and written once)
     append_gbs = append_bytes / (statistics.fmean(append_ms) * 1e-3) / 1e9
-    cache_bytes_read = 2 * (w.kv_len - w.chunk_len) * w.batch * w.heads * w.head_dim * 2
     line = {
         "metric": METRIC,
         "value": value,
@@ -556,19 +574,7 @@ def run_ours(args, w):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {
-            "workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
-            "chunk_tokens": w.chunk_len, "kv_tokens": w.kv_len, "sink_chunks": w.sink,
-            "window_chunks": w.window, "denoise_steps_per_chunk": w.steps, "layers": w.layers,
-            "step": "all denoising attentions of one chunk (every layer) + noisy and clean appends",
-            "l2": f"inputs larger than L2: {cache_bytes_read / 2**20:.0f} MiB of cached K/V "
-                  f"read per attention vs {L2_BYTES / 2**20:.0f} MiB L2",
-            "parallelism": (f"ulysses{world}-{args.transport}" if args.ulysses else
-                            f"replicas{world}" if world > 1 else "single"),
-            "block_sparsity": args.sparsity,
-            "ref_frames": args.ref_frames, "ref_tokens": ref_len,
-            "frame_aligned_editing": args.editing,
-        },
+        "config": workload_config(w, args, world),
         "roofline": {
             "bound": "tensor",
             "kernel": "attend_tc_kernel<128>" + (
