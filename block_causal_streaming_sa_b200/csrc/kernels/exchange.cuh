@@ -15,10 +15,11 @@
 // sender's pack made it) -> y: split 1: [B][G*T'][C'][D] (token shards in rank
 // order); split 0: [B][T'][G*C'][D] (head groups in rank order).
 //
-// fp8 (e4m3) with one scale per (b, t, c) vector: scale = max|x| / 448, code =
-// e4m3(x / scale), nearest even and saturated; on arrival code * scale in fp32,
-// rounded to bf16. The divisions are IEEE fp32 (div.rn), so the codes do not
-// depend on how the quotient is approximated.
+// fp8 (e4m3) with one scale per (b, t, c) vector: scale = max|x| / 448 and
+// inv = 448 / max|x| (one IEEE fp32 division each per vector), code =
+// e4m3(x * inv), nearest even and saturated; on arrival code * scale in fp32,
+// rounded to bf16. Every operation is a single IEEE fp32 one (div.rn, mul.rn),
+// so the codes do not depend on how a quotient is approximated.
 #pragma once
 
 #include <cstdint>
@@ -105,13 +106,26 @@ __global__ void __launch_bounds__(256) exchange_pack_kernel(ExchangeParams p) {
       w[k][0] = *reinterpret_cast<const uint32_t*>(src);
     }
   }
+  // (b, t, c) of the first vector once (64-bit division is a long routine),
+  // then stepped for the next ones
+  int c = 0, t = 0, b = 0;
+  if (vec0 < n_vec) {
+    c = static_cast<int>(vec0 % p.C);
+    const long long bt = vec0 / p.C;
+    t = static_cast<int>(bt % p.T);
+    b = static_cast<int>(bt / p.T);
+  }
 #pragma unroll
   for (int k = 0; k < V; ++k) {
     const long long vec = vec0 + k;
     if (vec >= n_vec) break;
-    const int c = static_cast<int>(vec % p.C);
-    const long long bt = vec / p.C;
-    const int t = static_cast<int>(bt % p.T), b = static_cast<int>(bt / p.T);
+    if (k > 0 && ++c == p.C) {
+      c = 0;
+      if (++t == p.T) {
+        t = 0;
+        ++b;
+      }
+    }
     int g;
     long long v;
     exchange_place(p, b, t, c, g, v);
@@ -136,11 +150,12 @@ __global__ void __launch_bounds__(256) exchange_pack_kernel(ExchangeParams p) {
     for (int off = 16; off > 0; off >>= 1)
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     const float scale = __fdiv_rn(amax, kE4m3Max);
+    const float inv = amax > 0.f ? __fdiv_rn(kE4m3Max, amax) : 0.f;
     uint8_t* codes = blk + v * D + lane * E;
     uint16_t q[E / 2];
 #pragma unroll
     for (int i = 0; i < E / 2; ++i)
-      q[i] = scale > 0.f ? e4m3x2(__fdiv_rn(f[2 * i], scale), __fdiv_rn(f[2 * i + 1], scale))
+      q[i] = scale > 0.f ? e4m3x2(__fmul_rn(f[2 * i], inv), __fmul_rn(f[2 * i + 1], inv))
                          : static_cast<uint16_t>(0);
     if constexpr (E == 4)
       *reinterpret_cast<uint32_t*>(codes) = static_cast<uint32_t>(q[0]) |
@@ -166,13 +181,24 @@ __global__ void __launch_bounds__(256) exchange_unpack_kernel(ExchangeParams p) 
   const long long n_vec = static_cast<long long>(p.B) * Ty * Cy;
   uint32_t raw[V][E / 2];  // bf16 words, or the E code bytes in raw[k][0] (fp8)
   float scale[V];
+  int cy = 0, ty = 0, b = 0;  // of the first vector once, then stepped (as in pack)
+  if (vec0 < n_vec) {
+    cy = static_cast<int>(vec0 % Cy);
+    const long long bt = vec0 / Cy;
+    ty = static_cast<int>(bt % Ty);
+    b = static_cast<int>(bt / Ty);
+  }
 #pragma unroll
   for (int k = 0; k < V; ++k) {
     const long long vec = vec0 + k;
     if (vec >= n_vec) break;
-    const int cy = static_cast<int>(vec % Cy);
-    const long long bt = vec / Cy;
-    const int ty = static_cast<int>(bt % Ty), b = static_cast<int>(bt / Ty);
+    if (k > 0 && ++cy == Cy) {
+      cy = 0;
+      if (++ty == Ty) {
+        ty = 0;
+        ++b;
+      }
+    }
     int s, tl = ty, cl = cy;
     if (p.split == 1) {
       s = ty / Tb;

@@ -316,8 +316,9 @@ SA_API int sa_stream_plan(const sa_handle* h, int step_is_final, int n_frames, i
  * token; split_dim 0 (tokens, after attention): block g holds tokens g*T/G ..
  * with every head. The split dimension must be a multiple of G.
  * Payload SA_PAYLOAD_FP8: each (b, t, c) vector of D values is sent as fp8
- * e4m3 codes (scale = max|x| / 448, code = e4m3(x / scale), nearest even,
- * saturating; IEEE fp32 division) followed by its fp32 scale, D + 4 bytes
+ * e4m3 codes (scale = max|x| / 448, inv = 448 / max|x|, code = e4m3(x * inv),
+ * nearest even, saturating; each an IEEE fp32 operation) followed by its fp32
+ * scale, D + 4 bytes
  * instead of 2 D; on arrival code * scale (fp32) rounded to bf16. An all-zero
  * vector has scale 0. SA_PAYLOAD_BF16 sends the values unchanged. Inputs must
  * be finite.

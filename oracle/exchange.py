@@ -19,11 +19,12 @@ all-to-all brings the output back to token shards with all heads.
 Reading R16 (the pages give no format): the exchanged payload is fp8 e4m3
 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; no infinities; largest
 finite 448) with one fp32 scale per (batch, token, head) vector of D values:
-scale = max|x| / 448 in fp32, code = e4m3(x / scale) rounded to nearest even
-and saturated to +-448, value on arrival = code * scale in fp32, rounded to
-bf16 (nearest even). An all-zero vector has scale 0 and codes 0. Inputs are
-finite. Divisions and products are fp32 (IEEE), so the integer codes are
-decided in the same precision on both sides.
+scale = max|x| / 448 and inv = 448 / max|x| (each one fp32 division per
+vector), code = e4m3(x * inv) rounded to nearest even and saturated to +-448,
+value on arrival = code * scale in fp32, rounded to bf16 (nearest even). An
+all-zero vector has scale 0 and codes 0. Inputs are finite. Every division and
+product is one IEEE fp32 operation, so the integer codes are decided in the
+same precision on both sides.
 """
 
 import numpy as np
@@ -74,8 +75,9 @@ def quantize(x):
     x32 = np.asarray(x, dtype=np.float32)
     amax = np.abs(x32).max(axis=-1)
     scale = (amax / np.float32(E4M3_MAX)).astype(np.float32)
-    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
-    q = (x32 / safe[..., None]).astype(np.float32)
+    safe = np.where(amax > 0, amax, np.float32(1.0)).astype(np.float32)
+    inv = (np.float32(E4M3_MAX) / safe).astype(np.float32)
+    q = (x32 * inv[..., None]).astype(np.float32)
     codes = e4m3_encode(q)
     codes = np.where(scale[..., None] > 0, codes, np.uint8(0)).astype(np.uint8)
     return codes, scale
