@@ -19,7 +19,14 @@
  *      abbreviation table - the KV cache stores history keys and values so they
  *      are not recomputed; RoPE encodes each token's position in space and time.
  *      section 2.2 - block-wise causal mask, anchor chunks, sliding-window
- *      context, noisy KV cache.
+ *      context, noisy KV cache, a reference image shared by every segment.
+ *      section 2.4 - multi-GPU Ulysses context parallelism with quantised
+ *      inter-GPU tensors; section 2.6 - the editing model's frame-aligned
+ *      attention.
+ *  The extensions cite their sections at each call: reference image and chunk
+ *  length (sa_set_reference, sa_append_chunk_frames), block sparsity
+ *  (sa_attend_sparse), frame-aligned editing (sa_attend_aligned), Ulysses
+ *  exchange (sa_exchange_*).
  *
  * Conventions shared by every call
  *  - Tensors are bfloat16, row-major [B, L, H, D] (batch, token of the chunk,
@@ -29,8 +36,8 @@
  *  - K and V passed in are UNROTATED; the library applies the 3D RoPE.
  *  - All device work is asynchronous on the caller's stream (a cudaStream_t
  *    passed as sa_stream; NULL is the legacy default stream). After sa_create,
- *    sa_append_chunk / sa_stage_keys / sa_attend_staged / sa_attend allocate no
- *    memory and never synchronise the host.
+ *    the append, reference, staging and attention calls allocate no memory and
+ *    never synchronise the host (sa_reset and sa_get_status do synchronise).
  *  - The device calls can be captured into a CUDA graph. A captured attention
  *    keeps the plan of the chunk it was captured for (attended chunks, slots
  *    and relocated positions are launch arguments): replay it for that chunk's
