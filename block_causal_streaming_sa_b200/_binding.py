@@ -79,6 +79,7 @@ _SIGNATURES = {
     "sa_block_grid": (_I, [_CFGP, ctypes.c_int32, _I32P, _I32P]),
     "sa_debug_attend_stalled": (_I, [_P, _P, _P, _P, _I, _P, _P]),
     "sa_chunk_count": (_I, [_P, _I]),
+    "sa_debug_inject_cuda_error": (_I, [_P]),
     "sa_debug_layout": (_I, [_P, _I, _I32P, _I]),
     "sa_plan": (_I, [_CFGP, ctypes.c_int32, _I32P, _I32P, _I32P, _I]),
     "sa_stream_plan": (_I, [_P, _I, _I, _I32P, _I32P, _I32P, _I]),
@@ -236,6 +237,11 @@ def sa_debug_attend_stalled(handle, Q, Kc, Vc, step_is_final, O, stream=0):
 
 def sa_debug_exp2(use_polynomial, x, y, n, stream=0):
     _check(lib().sa_debug_exp2(int(bool(use_polynomial)), _P(x), _P(y), int(n), _P(stream)))
+
+
+def sa_debug_inject_cuda_error(handle):
+    """Make the handle's next launching call fail with SA_ERR_CUDA (test hook)."""
+    _check(lib().sa_debug_inject_cuda_error(handle), handle)
 
 
 def sa_chunk_count(handle, tier):

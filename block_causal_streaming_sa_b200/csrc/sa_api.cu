@@ -14,6 +14,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "sa_internal.h"
 #include "kernels/attend_simt.cuh"
 #include "kernels/attend_tc.cuh"
@@ -28,6 +30,15 @@ using sa::RopeTables;
 namespace {
 
 thread_local std::string g_error;
+
+// NVTX range over one entry point (visible in Nsight timelines; a no-op
+// without a tool attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -288,6 +299,7 @@ struct sa_handle {
   bool staged_source;              // source-frame keys staged beside them
   bool has_cache;
   bool has_ref;  // a reference image is set
+  bool inject_cuda_error;  // test hook: the next launching call fails with SA_ERR_CUDA
   CUtensorMap tm_tier[2];
   CUtensorMap tm_kcur;
   CUtensorMap tm_ref;
@@ -323,6 +335,10 @@ int check_device(sa_handle* h) {
   if (cudaGetDevice(&dev) != cudaSuccess) return h->fail(SA_ERR_CUDA, "cudaGetDevice failed");
   if (dev != h->device)
     return h->fail(SA_ERR_INVALID_ARG, "current device differs from the handle's device");
+  if (h->inject_cuda_error) {  // test hook (sa_debug_inject_cuda_error)
+    h->inject_cuda_error = false;
+    return h->fail(SA_ERR_CUDA, "injected CUDA error (test hook)");
+  }
   return SA_OK;
 }
 
@@ -785,6 +801,7 @@ SA_API size_t sa_exchange_block_bytes(int B, int T, int C, int D, int G, int spl
 
 SA_API int sa_exchange_pack(const void* x, int B, int T, int C, int D, int G, int split_dim,
                             int payload, void* buf, sa_stream stream) {
+  NvtxRange range_("sa_exchange_pack");
   sa::ExchangeParams ep;
   if (!exchange_layout(B, T, C, D, G, split_dim, payload, &ep)) return SA_ERR_INVALID_ARG;
   if (x == nullptr || buf == nullptr || !aligned16(x) || !aligned16(buf)) {
@@ -798,6 +815,7 @@ SA_API int sa_exchange_pack(const void* x, int B, int T, int C, int D, int G, in
 
 SA_API int sa_exchange_pack_to(const void* x, int B, int T, int C, int D, int G, int split_dim,
                                int payload, void* const* dst_blocks, sa_stream stream) {
+  NvtxRange range_("sa_exchange_pack_to");
   sa::ExchangeParams ep;
   if (!exchange_layout(B, T, C, D, G, split_dim, payload, &ep)) return SA_ERR_INVALID_ARG;
   if (G > sa::kMaxExchangeRanks) {
@@ -888,6 +906,7 @@ SA_API int sa_ipc_close(void* dev_ptr) {
 
 SA_API int sa_exchange_unpack(const void* buf, int B, int T, int C, int D, int G, int split_dim,
                               int payload, void* y, sa_stream stream) {
+  NvtxRange range_("sa_exchange_unpack");
   sa::ExchangeParams ep;
   if (!exchange_layout(B, T, C, D, G, split_dim, payload, &ep)) return SA_ERR_INVALID_ARG;
   if (y == nullptr || buf == nullptr || !aligned16(y) || !aligned16(buf) || y == buf) {
@@ -965,6 +984,7 @@ SA_API int sa_create(const sa_config* cfg, void* dev_buf, size_t bytes, sa_handl
   h->staged_frames = d.F;
   h->staged_source = false;
   h->has_ref = false;
+  h->inject_cuda_error = false;
 
   // RoPE tables: angle pos * theta^(-2i/d) in double, cos/sin cast to float.
   // Temporal positions run over the reference frames and S + W chunks.
@@ -1053,16 +1073,19 @@ SA_API int sa_reset(sa_handle* h) {
 
 SA_API int sa_append_chunk(sa_handle* h, int tier, const void* K, const void* V,
                            sa_stream stream) {
+  NvtxRange range_("sa_append_chunk");
   if (h == nullptr) return check_handle(h);
   return append_chunk(h, tier, K, V, h->d.F, stream);
 }
 
 SA_API int sa_append_chunk_frames(sa_handle* h, int tier, const void* K, const void* V,
                                   int n_frames, sa_stream stream) {
+  NvtxRange range_("sa_append_chunk_frames");
   return append_chunk(h, tier, K, V, n_frames, stream);
 }
 
 SA_API int sa_set_reference(sa_handle* h, const void* K, const void* V, sa_stream stream) {
+  NvtxRange range_("sa_set_reference");
   int rc = check_handle(h);
   if (rc != SA_OK) return rc;
   if (K == nullptr && V == nullptr) {
@@ -1084,6 +1107,7 @@ SA_API int sa_set_reference(sa_handle* h, const void* K, const void* V, sa_strea
 
 SA_API int sa_attend(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
                      int step_is_final, void* O, float* lse, sa_stream stream) {
+  NvtxRange range_("sa_attend");
   if (h == nullptr) return check_handle(h);
   return attend_common(h, Q, Kc, Vc, h->d.F, step_is_final, O, lse, stream, false);
 }
@@ -1091,26 +1115,31 @@ SA_API int sa_attend(sa_handle* h, const void* Q, const void* Kc, const void* Vc
 SA_API int sa_attend_frames(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
                             int n_frames, int step_is_final, void* O, float* lse,
                             sa_stream stream) {
+  NvtxRange range_("sa_attend_frames");
   return attend_common(h, Q, Kc, Vc, n_frames, step_is_final, O, lse, stream, false);
 }
 
 SA_API int sa_attend_aligned(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
                              const void* Ks, const void* Vs, int n_frames, int step_is_final,
                              void* O, float* lse, sa_stream stream) {
+  NvtxRange range_("sa_attend_aligned");
   return attend_aligned(h, Q, Kc, Vc, Ks, Vs, n_frames, step_is_final, O, lse, stream);
 }
 
 SA_API int sa_stage_keys(sa_handle* h, const void* Kc, sa_stream stream) {
+  NvtxRange range_("sa_stage_keys");
   if (h == nullptr) return check_handle(h);
   return stage_keys(h, Kc, h->d.F, stream);
 }
 
 SA_API int sa_stage_keys_frames(sa_handle* h, const void* Kc, int n_frames, sa_stream stream) {
+  NvtxRange range_("sa_stage_keys_frames");
   return stage_keys(h, Kc, n_frames, stream);
 }
 
 SA_API int sa_attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final,
                             void* O, float* lse, sa_stream stream) {
+  NvtxRange range_("sa_attend_staged");
   return attend_staged(h, Q, Vc, step_is_final, O, lse, stream, false);
 }
 
@@ -1122,12 +1151,14 @@ SA_API int sa_debug_attend_simt(sa_handle* h, const void* Q, const void* Kc, con
 
 SA_API int sa_attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
                              int step_is_final, void* O, float* lse, sa_stream stream) {
+  NvtxRange range_("sa_attend_noalloc");
   return attend_noalloc(h, Q, Kc, Vc, step_is_final, O, lse, stream);
 }
 
 SA_API int sa_attend_sparse(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
                             int step_is_final, const uint8_t* block_mask, void* O, float* lse,
                             sa_stream stream) {
+  NvtxRange range_("sa_attend_sparse");
   int rc = check_handle(h);
   if (rc != SA_OK) return rc;
   if (block_mask == nullptr) return h->fail(SA_ERR_INVALID_ARG, "block_mask must be non-NULL");
@@ -1170,6 +1201,13 @@ SA_API int sa_debug_exp2(int use_polynomial, const float* x, float* y, int n, sa
     g_error = std::string("exp2 probe launch: ") + cudaGetErrorString(e);
     return SA_ERR_CUDA;
   }
+  return SA_OK;
+}
+
+SA_API int sa_debug_inject_cuda_error(sa_handle* h) {
+  int rc = check_handle(h);
+  if (rc != SA_OK) return rc;
+  h->inject_cuda_error = true;
   return SA_OK;
 }
 

@@ -283,6 +283,12 @@ SA_API int sa_debug_attend_stalled(sa_handle* h, const void* Q, const void* Kc, 
  * hook for the kernel's arithmetic; asynchronous on `stream`. */
 SA_API int sa_debug_exp2(int use_polynomial, const float* x, float* y, int n, sa_stream stream);
 
+/* Test hook for the host error path: the next call of this handle that would
+ * launch device work fails with SA_ERR_CUDA before launching anything (as a
+ * failed CUDA call would), leaving the handle's state unchanged; later calls
+ * work again. No device work, no fault. */
+SA_API int sa_debug_inject_cuda_error(sa_handle* h);
+
 /* Chunks appended so far to `tier`, or a negative sa_status. */
 SA_API int sa_chunk_count(const sa_handle* h, int tier);
 
