@@ -44,7 +44,11 @@
 //  * work units: rounds of gridDim.x work tiles; when the last round holds at
 //    most half a grid of tiles, each of them is split by attended chunks into
 //    two halves run by two CTAs, which write normalised fp32 partial rows and
-//    their log-sum-exp; per row, the second half to finish merges both.
+//    their log-sum-exp; per row, the second half to finish merges both;
+//  * block-sparse: the mask arrives as bit rows (one per query tile); step j of
+//    a work tile loads and multiplies the j-th flagged key tile of each of its
+//    two query tiles, so the ping-pong of the dense loop is kept (a key tile
+//    both flag at the same step is loaded once).
 // All mbarrier waits are bounded (see ptx.cuh); on a timeout every role drains
 // its outstanding async work, TMEM is freed and the device status word is set.
 #pragma once
@@ -235,7 +239,6 @@ __global__ void __launch_bounds__(384, 1)
   using T = TcShape<D>;
   constexpr bool kSparse = kMode == kModeSparse;    // caller-flagged 128 x 128 blocks
   constexpr bool kAligned = kMode == kModeAligned;  // last group: same-frame source keys
-  constexpr bool kSkip = kMode != kModeDense;       // some key tiles of a unit are skipped
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = ptx::smem_addr(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -318,19 +321,12 @@ __global__ void __launch_bounds__(384, 1)
   auto g_lo = [&](int half) { return half == 1 ? sched[3] : 0; };
   auto g_hi = [&](int half) { return half == 0 ? sched[3] : p.n_groups; };
 
-  // Skipped key tiles. Block sparsity: key tile kt of a work tile is visited
-  // when either of its two query tiles has the block flagged; flag rows at mask
-  // offsets mo (query tile 2 * pair) and mo1 (its partner, -1 when the pair has a
-  // single tile). Frame-aligned: of the last group (the source frames), only the
-  // tiles [mo, mo1) holding the frames of the work tile's rows are visited; every
-  // other group is visited whole.
+  // Skipped key tiles, frame-aligned mode: of the last group (the source frames),
+  // only the tiles [mo, mo1) holding the frames of the work tile's rows are
+  // visited; every other group is visited whole.
   auto mask_rows = [&](int w, int& mo, int& mo1) {
     mo = mo1 = -1;
-    if constexpr (kSparse) {
-      const int bh = w / n_pairs, pair = w - bh * n_pairs;
-      mo = (bh * n_qt + 2 * pair) * n_kt_total;
-      mo1 = 2 * pair + 1 < n_qt ? mo + n_kt_total : -1;
-    } else if constexpr (kAligned) {
+    if constexpr (kAligned) {
       const int pair = w % n_pairs;
       const int hw = p.rope.frame_tokens;
       const int q0 = 2 * pair * T::BM, q1 = min(q0 + 2 * T::BM, p.L) - 1;
@@ -339,22 +335,35 @@ __global__ void __launch_bounds__(384, 1)
       mo1 = gstart[gs] + (min((q1 / hw + 1) * hw, groups[gs].len) + T::BN - 1) / T::BN;
     }
   };
-  auto flag = [&](int off, int kt) -> bool {
-    return off >= 0 && __ldg(p.block_mask + off + kt) != 0;
-  };
   // First visited flat key tile in [from, hi), or a value >= hi if none.
   auto next_visited = [&](int mo, int mo1, int from, int hi) {
-    if constexpr (kSparse) {
-      int kt = from;
-      while (kt < hi && !(flag(mo, kt) || flag(mo1, kt))) ++kt;
-      return kt;
-    } else if constexpr (kAligned) {
+    if constexpr (kAligned) {
       if (from < gstart[p.n_groups - 1]) return from;
       const int u = from < mo ? mo : from;
       return u < mo1 && u < hi ? u : hi;
     } else {
       return from;
     }
+  };
+
+  // Block sparsity: the flagged key tiles of query tile i of work tile w as a bit
+  // row (null when the pair has a single query tile), and the first flagged tile
+  // of a row in [from, hi), or hi when there is none.
+  const int n_words = (n_kt_total + 63) >> 6;
+  auto bit_row = [&](int w, int i) -> const unsigned long long* {
+    const int bh = w / n_pairs, q = 2 * (w - bh * n_pairs) + i;
+    return q < n_qt ? p.block_bits + (static_cast<size_t>(bh) * n_qt + q) * n_words : nullptr;
+  };
+  auto next_set = [&](const unsigned long long* row, int from, int hi) -> int {
+    if (row == nullptr || from >= hi) return hi;
+    int wd = from >> 6;
+    unsigned long long bits = __ldg(row + wd) & (~0ull << (from & 63));
+    while (bits == 0ull) {
+      if (++wd << 6 >= hi) return hi;
+      bits = __ldg(row + wd);
+    }
+    const int k = (wd << 6) + __ffsll(static_cast<long long>(bits)) - 1;
+    return k < hi ? k : hi;
   };
 
   if (warp < 4) {
@@ -370,58 +379,80 @@ __global__ void __launch_bounds__(384, 1)
       int stage = 0;
       uint32_t phase = 0, filled_mask = 0, filled_parity = 0;
       bool ok = true;
+      // K (kv 0) or V (kv 1) of key tile t of group grp into the next stage.
+      auto load_kv = [&](const AttendGroup grp, int b, int h, int t, int kv) -> bool {
+        if (!ptx::mbar_wait(bar(T::EMPTY(stage)), phase ^ 1u, abort_flag, p.status))
+          return false;
+        const uint32_t full = bar(T::FULL(stage));
+        ptx::mbar_arrive_expect_tx(full, T::kTile);
+        const uint32_t dst = sbase + T::kOffKV + stage * T::kTile;
+        for (int kb = 0; kb < T::KBLK; ++kb) {
+          if (grp.src == 0) {
+            const int plane = ((grp.slot * 2 + kv) * p.B + b) * p.H + h;
+            ptx::tma_load_3d(dst + kb * T::kBox, &tm_cache, full, kb * 64, t * T::BN, plane);
+          } else if (grp.src == 2) {
+            ptx::tma_load_3d(dst + kb * T::kBox, &tm_ref, full, kb * 64, t * T::BN,
+                             (kv * p.B + b) * p.H + h);
+          } else if (grp.src == 3) {  // source frames: keys in scratch half 1
+            if (kv == 0)
+              ptx::tma_load_3d(dst + kb * T::kBox, &tm_kcur, full, kb * 64, t * T::BN,
+                               (p.B + b) * p.H + h);
+            else
+              ptx::tma_load_4d(dst + kb * T::kBox, &tm_vsrc, full, kb * 64, h, t * T::BN, b);
+          } else if (kv == 0) {
+            ptx::tma_load_3d(dst + kb * T::kBox, &tm_kcur, full, kb * 64, t * T::BN,
+                             b * p.H + h);
+          } else {
+            ptx::tma_load_4d(dst + kb * T::kBox, &tm_vcur, full, kb * 64, h, t * T::BN, b);
+          }
+        }
+        filled_mask |= 1u << stage;
+        filled_parity = (filled_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == T::NSTAGE) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        return true;
+      };
       for (int rr = 0; ok; ++rr) {
         int w, half;
         if (!unit(rr, w, half)) break;
         const int bh = w / n_pairs;
         const int b = bh / p.H, h = bh - b * p.H;
-        int mo, mo1;
-        mask_rows(w, mo, mo1);
-        for (int g = g_lo(half); ok && g < g_hi(half); ++g) {
-          const AttendGroup grp = groups[g];
-          int t0 = 0, t1 = (grp.len + T::BN - 1) / T::BN;
-          if (kAligned && g == p.n_groups - 1) {
-            t0 = mo - gstart[g];
-            t1 = mo1 - gstart[g];
-          }
-          for (int t = t0; ok && t < t1; ++t) {
-            if (kSparse && !(flag(mo, gstart[g] + t) || flag(mo1, gstart[g] + t))) continue;
-            for (int kv = 0; kv < 2; ++kv) {
-              if (!ptx::mbar_wait(bar(T::EMPTY(stage)), phase ^ 1u, abort_flag, p.status)) {
-                ok = false;
-                break;
-              }
-              const uint32_t full = bar(T::FULL(stage));
-              ptx::mbar_arrive_expect_tx(full, T::kTile);
-              const uint32_t dst = sbase + T::kOffKV + stage * T::kTile;
-              for (int kb = 0; kb < T::KBLK; ++kb) {
-                if (grp.src == 0) {
-                  const int plane = ((grp.slot * 2 + kv) * p.B + b) * p.H + h;
-                  ptx::tma_load_3d(dst + kb * T::kBox, &tm_cache, full, kb * 64, t * T::BN, plane);
-                } else if (grp.src == 2) {
-                  ptx::tma_load_3d(dst + kb * T::kBox, &tm_ref, full, kb * 64, t * T::BN,
-                                   (kv * p.B + b) * p.H + h);
-                } else if (grp.src == 3) {  // source frames: keys in scratch half 1
-                  if (kv == 0)
-                    ptx::tma_load_3d(dst + kb * T::kBox, &tm_kcur, full, kb * 64, t * T::BN,
-                                     (p.B + b) * p.H + h);
-                  else
-                    ptx::tma_load_4d(dst + kb * T::kBox, &tm_vsrc, full, kb * 64, h, t * T::BN,
-                                     b);
-                } else if (kv == 0) {
-                  ptx::tma_load_3d(dst + kb * T::kBox, &tm_kcur, full, kb * 64, t * T::BN,
-                                   b * p.H + h);
-                } else {
-                  ptx::tma_load_4d(dst + kb * T::kBox, &tm_vcur, full, kb * 64, h, t * T::BN, b);
-                }
-              }
-              filled_mask |= 1u << stage;
-              filled_parity = (filled_parity & ~(1u << stage)) | (phase << stage);
-              if (++stage == T::NSTAGE) {
-                stage = 0;
-                phase ^= 1u;
-              }
+        if constexpr (kSparse) {
+          // Step j of a unit: the K tiles, then the V tiles, of the j-th flagged key
+          // tile of each query tile (one tile when the two coincide).
+          const int lo = gstart[g_lo(half)], hi = gstart[g_hi(half)];
+          const unsigned long long* r0 = bit_row(w, 0);
+          const unsigned long long* r1 = bit_row(w, 1);
+          int ta = next_set(r0, lo, hi), tb = next_set(r1, lo, hi);
+          int ga = g_lo(half), gb = ga;
+          while (ok && (ta < hi || tb < hi)) {
+            while (ta < hi && ta >= gstart[ga + 1]) ++ga;
+            while (tb < hi && tb >= gstart[gb + 1]) ++gb;
+            for (int kv = 0; ok && kv < 2; ++kv) {
+              if (ta < hi) ok = load_kv(groups[ga], b, h, ta - gstart[ga], kv);
+              if (ok && tb < hi && tb != ta) ok = load_kv(groups[gb], b, h, tb - gstart[gb], kv);
             }
+            ta = next_set(r0, ta + 1, hi);
+            tb = next_set(r1, tb + 1, hi);
+          }
+        } else {
+          int mo, mo1;
+          mask_rows(w, mo, mo1);
+          for (int g = g_lo(half); ok && g < g_hi(half); ++g) {
+            const AttendGroup grp = groups[g];
+            int t0 = 0, t1 = (grp.len + T::BN - 1) / T::BN;
+            if (kAligned && g == p.n_groups - 1) {
+              t0 = mo - gstart[g];
+              t1 = mo1 - gstart[g];
+            }
+            for (int t = t0; ok && t < t1; ++t)
+              for (int kv = 0; kv < 2; ++kv)
+                if (!load_kv(grp, b, h, t, kv)) {
+                  ok = false;
+                  break;
+                }
           }
         }
       }
@@ -473,7 +504,7 @@ __global__ void __launch_bounds__(384, 1)
         int mo, mo1;
         mask_rows(w, mo, mo1);
         int u = next_visited(mo, mo1, lo, hi);
-        if (kSkip && u >= hi) {  // no block flagged: nothing to multiply
+        if (kAligned && u >= hi) {  // no key tile: nothing to multiply
           for (int i = 0; i < 2 && ok; ++i)
             ok = ptx::mbar_wait(bar(T::QREADY(i)), rr & 1, abort_flag, p.status);
           continue;
@@ -520,12 +551,27 @@ __global__ void __launch_bounds__(384, 1)
             u = nu;
           }
         } else {
-          // Block-sparse: query tile i takes part in key tile t when its block is
-          // flagged (S, softmax and P.V for that tile only); the key stream is the
-          // union of both tiles' blocks.
-          auto wants = [&](int i, int t) { return flag(i == 0 ? mo : mo1, t); };
-          int sk = 0, sv = 0;
-          if (!take_stage(sk)) break;
+          // Block-sparse, in the producer's order: step j multiplies the j-th flagged
+          // key tile of each query tile, so the two softmax warpgroups alternate as
+          // in the dense loop; a query tile with fewer blocks drops out early.
+          const unsigned long long* r0 = bit_row(w, 0);
+          const unsigned long long* r1 = bit_row(w, 1);
+          int ta = next_set(r0, lo, hi), tb = next_set(r1, lo, hi);
+          // Stages of the tiles a (query tile 0) and c (query tile 1) of one step,
+          // -1 for none; one stage when a == c.
+          auto take_pair = [&](int a, int c, int& s0, int& s1) -> bool {
+            s0 = s1 = -1;
+            if (a < hi && !take_stage(s0)) return false;
+            if (c < hi) {
+              if (c == a)
+                s1 = s0;
+              else if (!take_stage(s1))
+                return false;
+            }
+            return true;
+          };
+          int sk0, sk1;
+          if (!take_pair(ta, tb, sk0, sk1)) break;
           ptx::tc_fence_after();
           for (int i = 0; i < 2; ++i) {
             if (!ptx::mbar_wait(bar(T::QREADY(i)), rr & 1, abort_flag, p.status)) {
@@ -533,24 +579,27 @@ __global__ void __launch_bounds__(384, 1)
               break;
             }
             ptx::tc_fence_after();
-            if (wants(i, u)) {
+            const int sk = i == 0 ? sk0 : sk1;
+            if (sk >= 0) {
               issue_s(i, sk);
               ptx::umma_commit(bar(T::SFULL(i)));
             }
           }
           if (!ok) break;
-          ptx::umma_commit(bar(T::EMPTY(sk)));
+          if (sk0 >= 0) ptx::umma_commit(bar(T::EMPTY(sk0)));
+          if (sk1 >= 0 && sk1 != sk0) ptx::umma_commit(bar(T::EMPTY(sk1)));
           bool issued[2] = {false, false};  // a P.V of tile i issued in this unit
-          while (ok && u < hi) {
-            const int nu = next_visited(mo, mo1, u + 1, hi);
-            const bool has_next = nu < hi;
-            if (!take_stage(sv) || (has_next && !take_stage(sk))) {
+          while (ok && (ta < hi || tb < hi)) {
+            const int na = next_set(r0, ta + 1, hi), nb = next_set(r1, tb + 1, hi);
+            int sv0, sv1, nk0, nk1;
+            if (!take_pair(ta, tb, sv0, sv1) || !take_pair(na, nb, nk0, nk1)) {
               ok = false;
               break;
             }
             ptx::tc_fence_after();
             for (int i = 0; i < 2; ++i) {
-              if (wants(i, u)) {
+              const int sv = i == 0 ? sv0 : sv1;
+              if (sv >= 0) {
                 if (!ptx::mbar_wait(bar(T::PFULL(i)), pf_phase[i], abort_flag, p.status)) {
                   ok = false;
                   break;
@@ -559,22 +608,26 @@ __global__ void __launch_bounds__(384, 1)
                 ptx::tc_fence_after();
                 issue_pv(i, sv, issued[i]);
                 issued[i] = true;
+                if (i == 1 || sv0 != sv1) ptx::umma_commit(bar(T::EMPTY(sv)));
               }
-              if (i == 1) ptx::umma_commit(bar(T::EMPTY(sv)));  // V read by both P.V
-              // S of tile i's next key tile; its S region is free: the softmax has
-              // published P of its previous tile, whose P.V is issued before this.
-              if (has_next && wants(i, nu)) {
-                issue_s(i, sk);
+              // S of tile i's next flagged tile; its S region is free: the softmax
+              // has published P of the current one, whose P.V is issued above.
+              const int nk = i == 0 ? nk0 : nk1;
+              if (nk >= 0) {
+                issue_s(i, nk);
                 ptx::umma_commit(bar(T::SFULL(i)));
               }
             }
             if (!ok) break;
-            if (has_next) ptx::umma_commit(bar(T::EMPTY(sk)));
-            u = nu;
+            if (nk0 >= 0) ptx::umma_commit(bar(T::EMPTY(nk0)));
+            if (nk1 >= 0 && nk1 != nk0) ptx::umma_commit(bar(T::EMPTY(nk1)));
+            ta = na;
+            tb = nb;
           }
-          if (ok)  // O of a query tile with at least one block is final
-            for (int i = 0; i < 2; ++i)
-              if (issued[i]) ptx::umma_commit(bar(T::OFINAL(i)));
+          // O of both query tiles, also of one without a block: its warpgroup waits
+          // for this before it loads the next unit's query tile.
+          if (ok)
+            for (int i = 0; i < 2; ++i) ptx::umma_commit(bar(T::OFINAL(i)));
         }
       }
       // Every MMA issued so far must finish before TMEM is released.
@@ -609,20 +662,18 @@ __global__ void __launch_bounds__(384, 1)
       const int x = qr % p.rope.tok_w;
       const size_t row_off = ((static_cast<size_t>(b) * p.L + qr) * p.H + h) * D;
       const int glo = g_lo(half), ghi = g_hi(half);
-      int mo = -1, mo1 = -1, own = -1;
-      if (kSkip) {
-        mask_rows(w, mo, mo1);
-        own = i == 0 ? mo : mo1;
-      }
+      int mo = -1, mo1 = -1;
+      if (kAligned) mask_rows(w, mo, mo1);
       // First chunk with a key tile of this query tile (it is rotated for it).
-      // Sparse: the tiles flagged for this query tile only; frame-aligned units
-      // visit every group, the last one partly.
-      int g0 = glo;
+      // Sparse: the tiles flagged for this query tile only, cur being the next
+      // one; frame-aligned units visit every group, the last one partly.
+      // (The bit row and its end are re-derived where used: fewer live registers.)
+      int g0 = glo, cur = 0;
       bool any_tile = true;
       if (kSparse) {
-        const int u0 = next_visited(own, -1, gstart[glo], gstart[ghi]);
-        any_tile = u0 < gstart[ghi];
-        while (g0 + 1 < ghi && u0 >= gstart[g0 + 1]) ++g0;
+        cur = next_set(bit_row(w, i), gstart[glo], gstart[ghi]);
+        any_tile = cur < gstart[ghi];
+        while (g0 + 1 < ghi && cur >= gstart[g0 + 1]) ++g0;
       }
 
       // Rotated query tile for that chunk; the raw temporal chunks are kept in
@@ -651,7 +702,12 @@ __global__ void __launch_bounds__(384, 1)
           t1 = mo1 - gstart[g];
         }
         for (int t = t0; t < t1; ++t) {
-          if (kSparse && !flag(own, gstart[g] + t)) continue;
+          int nxt = 0;  // sparse: the flagged tile after this one (gstart[ghi]: none)
+          if constexpr (kSparse) {
+            if (cur >= gstart[g] + t1) break;  // the next one lies in a later chunk
+            t = cur - gstart[g];
+            nxt = next_set(bit_row(w, i), cur + 1, gstart[ghi]);
+          }
           if (!ptx::mbar_wait(bar(T::SFULL(i)), s_phase, abort_flag, p.status)) {
             ok = false;
             break;
@@ -749,9 +805,9 @@ __global__ void __launch_bounds__(384, 1)
           // tile's temporal band to that chunk's relocated offset first.
           int gn = g;
           if (kSparse) {
-            const int nu = next_visited(own, -1, gstart[g] + t + 1, gstart[ghi]);
-            if (nu < gstart[ghi] && nu >= gstart[g + 1])
-              while (gn + 1 < ghi && nu >= gstart[gn + 1]) ++gn;
+            if (nxt < gstart[ghi] && nxt >= gstart[g + 1])
+              while (gn + 1 < ghi && nxt >= gstart[gn + 1]) ++gn;
+            cur = nxt;
           } else if (t == t1 - 1 && g + 1 < ghi) {
             gn = g + 1;
           }
@@ -771,7 +827,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (!ok) break;
 
-      if (any_tile) {
+      if (any_tile || kSparse) {  // sparse: committed for a tile without blocks too
         if (!ptx::mbar_wait(bar(T::OFINAL(i)), o_units & 1, abort_flag, p.status)) break;
         ++o_units;
         ptx::tc_fence_after();

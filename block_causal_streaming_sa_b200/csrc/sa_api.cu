@@ -19,6 +19,7 @@
 #include "sa_internal.h"
 #include "kernels/attend_simt.cuh"
 #include "kernels/attend_tc.cuh"
+#include "kernels/block_bits.cuh"
 #include "kernels/exchange.cuh"
 #include "kernels/rope.cuh"
 
@@ -51,7 +52,9 @@ struct Derived {
   size_t ref_elems;    // B * H * Lref * D
   // byte offsets inside the device buffer
   size_t off_status, off_rope_t, off_rope_h, off_rope_w, off_tier[2], off_kcur, off_ref;
-  size_t off_split_o, off_split_lse, off_split_sem, split_sem_bytes, total;
+  size_t off_split_o, off_split_lse, off_split_sem, split_sem_bytes;
+  size_t off_bits, bits_bytes;  // block-sparse mask as bit rows
+  size_t total;
 };
 
 int validate(const sa_config* c, std::string* why) {
@@ -140,6 +143,13 @@ Derived derive(const sa_config& c) {
   d.off_split_sem = off;
   d.split_sem_bytes = static_cast<size_t>(sa::kMaxSplitSlots) * 2 * 128 * sizeof(int);
   off += align_up(d.split_sem_bytes, 1024);
+  // block-sparse bit rows: B * H * n_q_tiles rows of ceil(n_k_tiles / 64) words,
+  // at most (S + W) chunks of ceil(L / 128) key tiles (no reference, no source)
+  const size_t q_tiles = (static_cast<size_t>(d.L) + 127) / 128;
+  const size_t words = (static_cast<size_t>(d.S + d.W) * q_tiles + 63) / 64;
+  d.off_bits = off;
+  d.bits_bytes = static_cast<size_t>(d.B) * d.H * q_tiles * words * sizeof(unsigned long long);
+  off += align_up(d.bits_bytes, 1024);
   d.total = off;
   return d;
 }
@@ -546,7 +556,6 @@ int attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final
   fill_common(h, tier, h->staged_frames, aligned, Q, Vc, O, lse, &ap);
   ap.k_cur = h->kcur();
   ap.debug_stall_producer = debug_stall ? 1 : 0;
-  ap.block_mask = block_mask;
   ap.split_o = reinterpret_cast<float*>(h->buf + d.off_split_o);
   ap.split_lse = reinterpret_cast<float*>(h->buf + d.off_split_lse);
   ap.split_sem = reinterpret_cast<int*>(h->buf + d.off_split_sem);
@@ -565,6 +574,20 @@ int attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final
       return h->fail(SA_ERR_CUDA, "TMA descriptor for Vc / Vs failed");
     AttendMaps maps{h->has_cache ? &h->tm_tier[tier] : &h->tm_kcur, &h->tm_kcur, &tm_v,
                     d.RF > 0 ? &h->tm_ref : &h->tm_kcur, aligned ? &tm_vs : &tm_v};
+    if (block_mask != nullptr) {
+      // Pack the mask's rows for this launch's key groups into bit rows.
+      sa::BlockBitsParams bp;
+      bp.mask = block_mask;
+      bp.bits = reinterpret_cast<unsigned long long*>(h->buf + d.off_bits);
+      bp.n_k = 0;
+      for (int g = 0; g < ap.n_groups; ++g) bp.n_k += (ap.groups[g].len + 127) / 128;
+      bp.n_words = (bp.n_k + 63) / 64;
+      bp.rows = 1LL * d.B * d.H * ((ap.L + 127) / 128);
+      if (static_cast<size_t>(bp.rows) * bp.n_words * sizeof(unsigned long long) > d.bits_bytes)
+        return h->fail(SA_ERR_UNSUPPORTED, "block mask larger than the bit-row region");
+      sa::block_bits_kernel<<<static_cast<unsigned>((bp.rows + 7) / 8), 256, 0, s>>>(bp);
+      ap.block_bits = bp.bits;
+    }
     const int mode = block_mask != nullptr ? sa::kModeSparse
                      : aligned             ? sa::kModeAligned
                                            : sa::kModeDense;

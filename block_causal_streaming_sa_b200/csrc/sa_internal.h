@@ -79,8 +79,11 @@ struct AttendParams {
   float scale_log2;  // softmax scale * log2(e)
   RopeTables rope;
   unsigned* status;
-  const uint8_t* block_mask;  // optional [B][H][n_q_tiles][n_k_tiles]: nonzero = the 128x128
-                              // block is attended; null = dense
+  // Block-sparse mode: the caller's [B][H][n_q_tiles][n_k_tiles] mask as bit rows,
+  // row (b * H + h) * n_q_tiles + q of ceil(n_k_tiles / 64) words, bit k % 64 of
+  // word k / 64 set when key tile k (over every attended group, in order) is
+  // attended by query tile q. Null in the other modes.
+  const unsigned long long* block_bits;
   // Split tail: when the last round of work tiles would leave most CTAs idle,
   // its tiles are split into two key-range halves; each half writes a
   // normalised fp32 partial row and its lse, and per row the second finisher

@@ -61,8 +61,33 @@ def test_structured_masks_skip_chunks_and_partner_tiles():
     m = np.zeros_like(masks[0])
     m[:, :, :, 2 * per_chunk:3 * per_chunk] = 1   # one middle chunk only
     masks.append(m)
+    m = np.zeros_like(masks[0])
+    m[:, :, 1::2, :] = 1                          # odd query tiles only: the first
+    masks.append(m)                               # tile of every pair sees nothing
+    rng = np.random.default_rng(3)
+    m = (rng.random(masks[0].shape) < 0.4).astype(np.uint8)
+    m[:, :, 1::2, :] = m[:, :, 0:nq - 1:2, :]     # both tiles of a pair alike: every
+    masks.append(m)                               # key tile is shared by the pair
     for i, m in enumerate(masks):
         _check(*pair.attend_sparse(0, True, m), f"structured mask {i}")
+
+
+@pytest.mark.parametrize("density", [0.02, 0.5])
+def test_rows_of_more_than_64_key_tiles(density):
+    """72 key tiles a query tile: the mask's bit rows span two words."""
+    w = Workload("sparse_wide", 1, 2, 128, 3, 16, 32, sink=1, window=5, steps=1, stream=6)
+    pair = Pair(w)
+    for _ in range(5):
+        pair.append()
+    nq, nk = _grid(pair)
+    assert nk > 64
+    rng = np.random.default_rng(int(density * 1000))
+    mask = (rng.random((w.batch, w.heads, nq, nk)) < density).astype(np.uint8)
+    mask[0, 0, 1, 60:70] = 1                      # a run across the word boundary
+    mask[0, 1, 2, :] = 0
+    mask[0, 1, 2, 64] = 1                         # a single block just past it
+    _check(*pair.attend_sparse(0, True, mask), f"wide rows density {density}")
+    assert pair.gpu.status() == sa.SA_OK
 
 
 def test_all_ones_mask_is_the_dense_kernel_bit_for_bit():
