@@ -591,8 +591,8 @@ __global__ void __launch_bounds__(384, 1)
           bool issued[2] = {false, false};  // a P.V of tile i issued in this unit
           while (ok && (ta < hi || tb < hi)) {
             const int na = next_set(r0, ta + 1, hi), nb = next_set(r1, tb + 1, hi);
-            int sv0, sv1, nk0, nk1;
-            if (!take_pair(ta, tb, sv0, sv1) || !take_pair(na, nb, nk0, nk1)) {
+            int sv0, sv1, nk0 = -1;
+            if (!take_pair(ta, tb, sv0, sv1)) {
               ok = false;
               break;
             }
@@ -611,16 +611,23 @@ __global__ void __launch_bounds__(384, 1)
                 if (i == 1 || sv0 != sv1) ptx::umma_commit(bar(T::EMPTY(sv)));
               }
               // S of tile i's next flagged tile; its S region is free: the softmax
-              // has published P of the current one, whose P.V is issued above.
-              const int nk = i == 0 ? nk0 : nk1;
-              if (nk >= 0) {
+              // has published P of the current one, whose P.V is issued above. Its
+              // K stage is taken only now: the ring holds one step, so the next
+              // step's K tiles may still be loading while this step's P.V runs.
+              const int nxt = i == 0 ? na : nb;
+              if (nxt < hi) {
+                int nk = nk0;
+                if ((i == 0 || nb != na) && !take_stage(nk)) {
+                  ok = false;
+                  break;
+                }
+                if (i == 0) nk0 = nk;
+                ptx::tc_fence_after();
                 issue_s(i, nk);
                 ptx::umma_commit(bar(T::SFULL(i)));
+                if (i == 1 || nb != na) ptx::umma_commit(bar(T::EMPTY(nk)));
               }
             }
-            if (!ok) break;
-            if (nk0 >= 0) ptx::umma_commit(bar(T::EMPTY(nk0)));
-            if (nk1 >= 0 && nk1 != nk0) ptx::umma_commit(bar(T::EMPTY(nk1)));
             ta = na;
             tb = nb;
           }
