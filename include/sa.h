@@ -100,8 +100,10 @@ SA_API int sa_validate_config(const sa_config* cfg);
  * a status word, fp32 RoPE tables, both cache tiers ((S + W - 1) slots of K and
  * V each, layout [slot][K|V][B][H][L][D], K fp16, V bf16), two rotated-key chunks of
  * scratch for the chunk being generated (its keys and, for sa_attend_aligned,
- * its source keys) and, when ref_frames > 0, the reference image
- * ([K|V][B][H][ref_frames * tok_h * tok_w][D]). Host only. */
+ * its source keys), when ref_frames > 0 the reference image
+ * ([K|V][B][H][ref_frames * tok_h * tok_w][D]), the split-tail scratch and
+ * the bit rows sa_attend_sparse packs its mask into (B * H * ceil(L / 128)
+ * rows of ceil((S + W) * ceil(L / 128) / 64) 64-bit words). Host only. */
 SA_API size_t sa_required_bytes(const sa_config* cfg);
 
 /* Create a handle over a caller-owned device buffer of at least
@@ -212,8 +214,12 @@ SA_API int sa_attend_aligned(sa_handle* h, const void* Q, const void* Kc, const 
  * chunk possibly short). block_mask: device uint8 [B][H][n_q_tiles][n_k_tiles]
  * (nonzero = attended); read only. n_k_tiles is the sum over the attended chunks
  * of ceil(keys / 128): sa_block_grid gives it when every chunk has F frames,
- * sa_stream_plan's lens in general. Key tiles no query tile of a 256-row pair
- * needs are neither loaded nor multiplied. A row that sees no key gets O = 0
+ * sa_stream_plan's lens in general. Three launches on the stream: the key
+ * staging of sa_stage_keys, the mask packed into bit rows in the handle's
+ * buffer (so block_mask may be rewritten once the call's work has run), and
+ * the attention. Only flagged blocks are loaded and multiplied (a key tile that
+ * both query tiles of a 256-row pair flag at the same step is loaded once).
+ * A row that sees no key gets O = 0
  * and lse = -inf. The reference image is not part of the block grid: with a
  * reference set this call returns SA_ERR_UNSUPPORTED. */
 SA_API int sa_attend_sparse(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
