@@ -57,7 +57,14 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
-    return ap.parse_args()
+    args = ap.parse_args()
+    if not 0.0 <= args.sparsity < 1.0:
+        ap.error("--sparsity must be in [0, 1)")
+    if sum((args.ulysses, args.editing, args.sparsity > 0)) > 1:
+        ap.error("--ulysses, --editing and --sparsity select different workloads; give one")
+    if args.sparsity > 0 and args.ref_frames > 0:
+        ap.error("block-sparse attention takes no reference image (--ref-frames 0)")
+    return args
 
 
 def attend_flops(w):
@@ -595,9 +602,11 @@ def run_ours(args, w):
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms_max / e2e_steps,
                 "pipelining": "inputs of step i+1 up and output of step i down on two copy "
                               "streams while step i computes"},
-        # per attention: stage + attend (+ 4 pack/unpack pairs with Ulysses);
-        # per append: one kernel (+ 2 pack/unpack pairs with Ulysses)
-        "gpu_launches": args.steps * ((10 if args.ulysses else 2) * attends_per_chunk
+        # per attention: stage + attend (+ the mask packing when block-sparse; + 4
+        # pack/unpack pairs with Ulysses); per append: one kernel (+ 2 pack/unpack
+        # pairs with Ulysses)
+        "gpu_launches": args.steps * ((10 if args.ulysses else 3 if args.sparsity > 0 else 2)
+                                      * attends_per_chunk
                                       + (5 if args.ulysses else 1) * appends_per_chunk),
         "clocks": clock_info,
         "cpu_baseline": cpu,

@@ -76,6 +76,19 @@ def test_reference_arm_line_on_rank_zero():
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
 
 
+@pytest.mark.parametrize("flags, why", [
+    (["--sparsity", "0.9", "--ulysses"], "different workloads"),
+    (["--editing", "--sparsity", "0.5"], "different workloads"),
+    (["--sparsity", "0.9", "--ref-frames", "1"], "no reference image"),
+    (["--sparsity", "1.0"], "must be in [0, 1)"),
+])
+def test_bench_refuses_mixed_workload_flags(flags, why):
+    """A mode flag the timed loop would ignore must not reach the FLOP count."""
+    r = subprocess.run([sys.executable, "bench.py", *flags], cwd=ROOT, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 2 and why in r.stderr, r.stderr
+
+
 def _a2a_worker(rank, world, port, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
