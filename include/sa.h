@@ -65,7 +65,7 @@ typedef enum {
   SA_OK = 0,
   SA_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or config field */
   SA_ERR_STATE = 2,        /* call not allowed in the handle's current state */
-  SA_ERR_UNSUPPORTED = 3,  /* valid request this build cannot serve (e.g. D) */
+  SA_ERR_UNSUPPORTED = 3,  /* valid request the library does not serve (e.g. D) */
   SA_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed */
   SA_ERR_TIMEOUT = 5       /* a kernel gave up a bounded wait (device status) */
 } sa_status;
@@ -89,7 +89,7 @@ typedef struct {
                                whether or not a reference is set. */
 } sa_config;
 
-/* Upper bounds of this build (checked by sa_validate_config). */
+/* Upper bounds of the library (checked by sa_validate_config). */
 #define SA_MAX_ATTENDED 16 /* S + W, and S + W + 1 when ref_frames > 0 */
 #define SA_MAX_CHUNK_LEN (1 << 22)
 
