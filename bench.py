@@ -167,39 +167,74 @@ def blas_threads():
 
 class OracleSample:
     """The float64 oracle on a bounded sample of the workload: the generating
-    chunk at steady state, one (batch, head) pair and a few query rows per call."""
+    chunk at steady state, one (batch, head) pair and a few query rows per call,
+    in the mode the bench line names (reference image, frame-aligned editing or
+    a block-sparse mask), with the same seeded inputs and mask as the GPU arm."""
 
-    def __init__(self, w):
+    def __init__(self, w, ref_frames=0, editing=False, sparsity=0.0):
         import numpy as np
         import torch
 
         from oracle.stream import CLEAN, NOISY, OracleConfig, StreamOracle
+        from sa_inputs import normal_bf16, seed_of
 
         self.np = np
         self.w = w
+        self.editing = editing
         cfg = OracleConfig(w.batch, w.heads, w.head_dim, w.frames, w.tok_h, w.tok_w, w.sink,
-                           w.window)
+                           w.window, ref_frames=ref_frames)
         self.orc = StreamOracle(cfg)
         f64 = lambda t: t.to(torch.float64).numpy()  # noqa: E731
+        hw = w.tok_h * w.tok_w
+        if ref_frames > 0:
+            shape = (w.batch, ref_frames * hw, w.heads, w.head_dim)
+            self.orc.set_reference(*(f64(normal_bf16(seed_of(w.name, "reference", n), shape))
+                                     for n in ("K", "V")))
         pool = [{n: f64(w.tensor(n, c)) for n in ("Kn", "Vn", "Kcl", "Vcl")} for c in range(2)]
         for c in range(w.sink + w.window - 1):
             s = pool[c % 2]
             self.orc.append(NOISY, s["Kn"], s["Vn"])
             self.orc.append(CLEAN, s["Kcl"], s["Vcl"])
-        self.cur = {n: f64(w.tensor(n, 9)) for n in ("Q", "Kc", "Vc")}
+        names = ("Q", "Kc", "Vc") + (("Ks", "Vs") if editing else ())
+        self.cur = {n: f64(w.tensor(n, 9)) for n in names}
+        # keys each query row sees (sparse: per query tile, from the mask)
+        self.row_keys = w.kv_len + ref_frames * hw + (hw if editing else 0)
+        self.mask = None
+        if sparsity > 0:
+            nq = -(-w.chunk_len // 128)
+            gen = torch.Generator().manual_seed(1234)
+            mask = torch.rand((w.batch, w.heads, nq, (w.sink + w.window) * nq), generator=gen)
+            self.mask = (mask >= sparsity).numpy()
+            tile_keys = np.full(nq, 128)
+            tile_keys[-1] = w.chunk_len - 128 * (nq - 1)
+            self.tile_row_keys = (self.mask * np.tile(tile_keys, w.sink + w.window)).sum(-1)
         self.rng = np.random.default_rng(3)
         self.calls = 0
+        self.mode = ("block-sparse" if sparsity > 0 else "frame-aligned editing" if editing
+                     else "dense") + (f", {ref_frames}-frame reference" if ref_frames else "")
 
     def run(self, rows):
         """One sample: `rows` query rows of one (b, h); returns its FLOPs."""
+        from oracle.editing import frame_aligned_attend
+        from oracle.sparse import block_sparse_attend
+
         w = self.w
         bh = self.calls % (w.batch * w.heads)
         self.calls += 1
         b, h = divmod(bh, w.heads)
         sel = self.rng.choice(w.chunk_len, size=rows, replace=False)
-        self.orc.attend(self.cur["Q"], self.cur["Kc"], self.cur["Vc"], True, rows=sel,
-                        heads=[h], batches=[b])
-        return 4.0 * rows * w.kv_len * w.head_dim
+        cur = self.cur
+        if self.mask is not None:
+            block_sparse_attend(self.orc, cur["Q"], cur["Kc"], cur["Vc"], True, self.mask,
+                                rows=sel, heads=[h], batches=[b])
+            return 4.0 * w.head_dim * float(self.tile_row_keys[b, h, sel // 128].sum())
+        if self.editing:
+            frame_aligned_attend(self.orc, cur["Q"], cur["Kc"], cur["Vc"], cur["Ks"], cur["Vs"],
+                                 True, rows=sel, heads=[h], batches=[b])
+        else:
+            self.orc.attend(cur["Q"], cur["Kc"], cur["Vc"], True, rows=sel, heads=[h],
+                            batches=[b])
+        return 4.0 * rows * self.row_keys * w.head_dim
 
     def calibrate(self, seconds):
         """Rows per call such that one call takes about `seconds`."""
@@ -214,8 +249,14 @@ class OracleSample:
         return int(min(self.w.chunk_len, max(16, (seconds - fixed) / per_row)))
 
 
-def cpu_baseline(w, seconds):
-    o = OracleSample(w)
+def oracle_sample(w, args):
+    return OracleSample(w, ref_frames=args.ref_frames, editing=args.editing,
+                        sparsity=args.sparsity)
+
+
+def cpu_baseline(w, args):
+    o = oracle_sample(w, args)
+    seconds = args.cpu_seconds
     rows = o.calibrate(min(seconds / 3, 5.0))
     flops, t0 = 0.0, time.perf_counter()
     while time.perf_counter() - t0 < seconds:
@@ -224,8 +265,8 @@ def cpu_baseline(w, seconds):
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
             "kind": "oracle",
             "sample": f"{o.calls - 2} calls x {rows} query rows of one (b,h) each, "
-                      f"all {w.kv_len} keys, final (clean-tier) step at steady state, "
-                      f"{dt:.1f} s of float64 numpy on the host"}
+                      f"{o.mode} attention over the chunk's keys, final (clean-tier) step "
+                      f"at steady state, {dt:.1f} s of float64 numpy on the host"}
 
 
 def workload_config(w, args, world):
@@ -251,7 +292,7 @@ def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    o = OracleSample(w)
+    o = oracle_sample(w, args)
     rows = o.calibrate(0.15)
     for _ in range(args.warmup):
         o.run(rows)
@@ -260,8 +301,8 @@ def run_reference(args, w):
         flops += o.run(rows)
     dt = time.perf_counter() - t0
     value = flops / dt / 1e12
-    sample = (f"each step: {rows} query rows of one (b,h) over all {w.kv_len} keys "
-              f"(float64 numpy oracle, host cores)")
+    sample = (f"each step: {rows} query rows of one (b,h), {o.mode} attention over the "
+              f"chunk's keys (float64 numpy oracle, host cores)")
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
@@ -554,7 +595,7 @@ def run_ours(args, w):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, args.cpu_seconds)
+        cpu = cpu_baseline(w, args)
 
     ranks.close()
     if rank != 0:

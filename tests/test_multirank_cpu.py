@@ -76,6 +76,42 @@ def test_reference_arm_line_on_rank_zero():
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
 
 
+@pytest.mark.parametrize("flags, key, mode", [
+    (["--sparsity", "0.5"], "block_sparsity", "block-sparse"),
+    (["--editing"], "frame_aligned_editing", "frame-aligned editing"),
+    (["--ref-frames", "1"], "ref_frames", "1-frame reference"),
+])
+def test_reference_arm_times_the_oracle_of_the_named_mode(flags, key, mode):
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny",
+                        "--steps", "1", "--warmup", "0", *flags], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["config"][key] and mode in line["cpu_baseline"]["sample"] and line["value"] > 0
+
+
+def test_oracle_sample_flops_follow_the_mode():
+    """FLOPs of a sampled call: 4 D x (keys each sampled row sees), as the GPU arm counts."""
+    import numpy as np
+
+    import bench
+    from sa_inputs import WORKLOADS
+
+    w = WORKLOADS["tiny"]
+    hw = w.tok_h * w.tok_w
+    assert bench.OracleSample(w).run(8) == 4.0 * 8 * w.kv_len * w.head_dim
+    assert bench.OracleSample(w, ref_frames=2).run(8) == 4.0 * 8 * (w.kv_len + 2 * hw) * w.head_dim
+    assert bench.OracleSample(w, editing=True).run(8) == 4.0 * 8 * (w.kv_len + hw) * w.head_dim
+    o = bench.OracleSample(w, sparsity=0.5)
+    o.rng = np.random.default_rng(0)
+    sel = np.random.default_rng(0).choice(w.chunk_len, size=8, replace=False)
+    nq = -(-w.chunk_len // 128)
+    tile = np.array([128, w.chunk_len - 128] * (w.sink + w.window))
+    keys = sum(int((o.mask[0, 0, q // 128] * tile).sum()) for q in sel)
+    assert o.run(8) == 4.0 * w.head_dim * keys and nq == 2
+
+
 @pytest.mark.parametrize("flags, why", [
     (["--sparsity", "0.9", "--ulysses"], "different workloads"),
     (["--editing", "--sparsity", "0.5"], "different workloads"),
