@@ -250,8 +250,11 @@ class OracleSample:
 
 
 def oracle_sample(w, args):
-    return OracleSample(w, ref_frames=args.ref_frames, editing=args.editing,
-                        sparsity=args.sparsity)
+    o = OracleSample(w, ref_frames=args.ref_frames, editing=args.editing,
+                     sparsity=args.sparsity)
+    if args.ulysses:
+        o.mode += " (the Ulysses layer's attention on all heads; its exchanges not sampled)"
+    return o
 
 
 def cpu_baseline(w, args):
