@@ -253,7 +253,7 @@ def oracle_sample(w, args):
     o = OracleSample(w, ref_frames=args.ref_frames, editing=args.editing,
                      sparsity=args.sparsity)
     if args.ulysses:
-        o.mode += " (the Ulysses layer's attention on all heads; its exchanges not sampled)"
+        o.mode += " (Ulysses layer: all heads, exchanges not sampled)"
     return o
 
 
