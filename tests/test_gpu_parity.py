@@ -5,7 +5,7 @@ import pytest
 import torch
 
 import block_causal_streaming_sa_b200 as sa
-from harness import TOL, Pair, check_output, f64, sample_rows
+from harness import TOL, Pair, check_output, sample_rows
 from oracle.stream import CLEAN, NOISY
 from sa_inputs import WORKLOADS, Workload
 

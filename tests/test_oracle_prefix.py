@@ -7,7 +7,6 @@ import pytest
 import torch
 
 from oracle import rope as orope
-from oracle.cache import RingCacheModel
 from oracle.stream import CLEAN, NOISY, OracleConfig, StreamOracle, masked_full_attention
 from sa_inputs import normal_bf16, seed_of
 
