@@ -38,6 +38,12 @@ def test_tiers_out_of_step_and_double_append_are_state_errors():
     assert e.value.status == sa.SA_ERR_STATE
     assert (h.chunk_count(NOISY), h.chunk_count(CLEAN)) == (1, 0)
     h.append(CLEAN, W.tensor("Kcl", 0).cuda(), W.tensor("Vcl", 0).cuda())
+    # the refused attention staged no keys either: its attention half alone is refused
+    Q, _, Vc = _tensors(1)
+    O = torch.empty_like(Q)
+    with pytest.raises(sa.SaError) as e:
+        sa.sa_attend_staged(h.handle, Q.data_ptr(), Vc.data_ptr(), False, O.data_ptr())
+    assert e.value.status == sa.SA_ERR_STATE
     h.attend(*_tensors(1), False)
     torch.cuda.synchronize()
     assert h.status() == sa.SA_OK
