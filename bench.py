@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 METRIC = "ms per chunk-step and attention TFLOP/s (% of B200 bf16 peak) at 720p shape"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 2 ** 20
+SUSTAINED_REGION_S = 2.0  # timed regions at least this long compare with the sustained peak
 
 
 def parse_args():
@@ -54,6 +55,9 @@ def parse_args():
                     help="frame-aligned editing attention (source frames of the chunk as extra keys)")
     ap.add_argument("--ref-frames", type=int, default=0,
                     help="frames of a reference image every chunk also attends (0: none)")
+    ap.add_argument("--launch-gaps", type=int, default=0, metavar="STEPS",
+                    help="after the timed region, trace STEPS more chunk-steps with the CUDA "
+                         "activity profiler and report the idle gaps between kernels")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
@@ -98,15 +102,41 @@ def kernel_traffic(kernel_file, workload):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples while the timed region runs."""
+    """SM clock, power and clock-event reasons sampled through NVML every ~2 ms
+    on a thread while the timed region runs (so a region of tens of ms still
+    gets tens of samples); ``stop`` keeps the samples taken between
+    ``mark_start`` and ``mark_stop`` (host times that bracket the device's
+    timed region). Falls back to ``nvidia-smi -lms`` when NVML is missing."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    # NVML clock-event reason bits of the four names above
+    BITS = (0x8, 0x40, 0x20, 0x4)
+    PERIOD_S = 0.002
 
     def __init__(self, bus_id):
+        import threading
+
+        self.samples = []  # (host time, sm MHz, max sm MHz, power W, reason bits)
+        self.t0 = self.t1 = None
         self.proc = None
+        self.nvml = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.dev = pynvml.nvmlDeviceGetHandleByPciBusId(bus_id)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.dev, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nvml = None
+        if self.nvml is not None:
+            self.halt = threading.Event()
+            self.thread = threading.Thread(target=self._loop, daemon=True)
+            self.thread.start()
+            return
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -115,34 +145,69 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
-    def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=10)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, smax, power, reasons = [], [], [], set()
-        for line in out.strip().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
+    def _loop(self):
+        n = self.nvml
+        reasons_fn = getattr(n, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            n.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.halt.is_set():
             try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-                power.append(float(parts[3]))
-            except ValueError:
-                continue
-            for name, val in zip(self.NAMES, parts[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
+                t = time.perf_counter()
+                sm = n.nvmlDeviceGetClockInfo(self.dev, n.NVML_CLOCK_SM)
+                power = n.nvmlDeviceGetPowerUsage(self.dev) / 1000.0
+                bits = reasons_fn(self.dev)
+                self.samples.append((t, float(sm), float(self.max_mhz), power, int(bits)))
+            except Exception:
+                pass
+            time.sleep(self.PERIOD_S)
+
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_stop(self):
+        self.t1 = time.perf_counter()
+
+    def stop(self):
+        if self.nvml is not None:
+            self.halt.set()
+            self.thread.join(timeout=5)
+            rows = [s for s in self.samples
+                    if (self.t0 is None or s[0] >= self.t0) and (self.t1 is None or s[0] <= self.t1)]
+            sm = [r[1] for r in rows]
+            smax = [r[2] for r in rows]
+            power = [r[3] for r in rows]
+            reasons = {name for r in rows for name, bit in zip(self.NAMES, self.BITS)
+                       if r[4] & bit}
+            source = "nvml"
+        elif self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=10)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            sm, smax, power, reasons = [], [], [], set()
+            for line in out.strip().splitlines():
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                    power.append(float(parts[3]))
+                except ValueError:
+                    continue
+                for name, val in zip(self.NAMES, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+            source = "nvidia-smi"
+        else:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"]}
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"],
+                    "source": source}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "power_w_median": statistics.median(power), "samples": len(sm),
-                "reasons": sorted(reasons)}
+                "sm_mhz_min": min(sm), "power_w_median": statistics.median(power),
+                "samples": len(sm), "source": source, "reasons": sorted(reasons)}
 
 
 def bus_id_of(dev):
@@ -319,6 +384,46 @@ def run_reference(args, w):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def launch_gap_trace(run_steps, n_steps):
+    """Kernel timeline of n_steps chunk-steps from the CUDA activity profiler
+    (CUPTI through torch.profiler; outside every timed region): busy time,
+    idle gaps between consecutive kernels, and time per kernel name."""
+    import tempfile
+
+    import torch
+    from torch.profiler import ProfilerActivity, profile
+
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        run_steps(n_steps)
+        torch.cuda.synchronize()
+    with tempfile.TemporaryDirectory() as d:
+        path = os.path.join(d, "trace.json")
+        prof.export_chrome_trace(path)
+        with open(path) as f:
+            events = json.load(f).get("traceEvents", [])
+    ks = sorted((float(e["ts"]), float(e["dur"]), e["name"]) for e in events
+                if e.get("cat") == "kernel")
+    if not ks:
+        return {"kernels": 0, "note": "the profiler recorded no kernel"}
+    gaps = [max(0.0, ks[i + 1][0] - (ks[i][0] + ks[i][1])) for i in range(len(ks) - 1)]
+    span = ks[-1][0] + ks[-1][1] - ks[0][0]
+    busy = sum(k[1] for k in ks)
+    per_name = {}
+    for _, dur, name in ks:
+        short = re.sub(r"\(.*", "", name)
+        c, t = per_name.get(short, (0, 0.0))
+        per_name[short] = (c + 1, t + dur)
+    q = statistics.quantiles(gaps, n=10) if len(gaps) >= 2 else [0.0] * 9
+    return {
+        "steps": n_steps, "kernels": len(ks), "span_ms": span / 1e3, "busy_ms": busy / 1e3,
+        "idle_ms": (span - busy) / 1e3, "idle_share": (span - busy) / span,
+        "gap_us": {"median": statistics.median(gaps) if gaps else 0.0, "p90": q[8],
+                   "max": max(gaps) if gaps else 0.0, "sum": sum(gaps)},
+        "by_kernel": {k: {"launches": c, "ms": t / 1e3} for k, (c, t) in per_name.items()},
+    }
 
 
 # ------------------------------------------------------------------ ranks
@@ -520,14 +625,18 @@ def run_ours(args, w):
         evs = [([mk() for _ in range(attends_per_chunk)], [mk() for _ in range(attends_per_chunk)],
                 mk(), mk()) for _ in range(args.steps)]
         start, stop = mk(), mk()
+        clocks = ClockSampler(bus_id_of(dev)) if rank == 0 else None
         barrier()
         torch.cuda.synchronize(dev)
-        clocks = ClockSampler(bus_id_of(dev)) if rank == 0 else None
+        if clocks is not None:
+            clocks.mark_start()
         start.record(stream)
         for i in range(args.steps):
             chunk_step(pool[i % 2], evs[i])
         stop.record(stream)
         stream.synchronize()
+        if clocks is not None:
+            clocks.mark_stop()
         torch.cuda.synchronize(dev)
         clock_info = clocks.stop() if clocks is not None else None
         barrier()
@@ -596,6 +705,14 @@ def run_ours(args, w):
     value = whole_job_tflops(flops_rank * attends_per_chunk * args.steps, ms_max, world)
     e2e_value = whole_job_tflops(flops_rank * attends_per_chunk * e2e_steps, e2e_ms_max, world)
 
+    gaps = None
+    if args.launch_gaps > 0 and world == 1:
+        def run_steps(n):
+            with torch.cuda.stream(stream):
+                for i in range(n):
+                    chunk_step(pool[i % 2])
+        gaps = launch_gap_trace(run_steps, args.launch_gaps)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args)
@@ -607,8 +724,25 @@ def run_ours(args, w):
     peaks, peak_src = load_peaks()
     attend_avg = statistics.fmean(attend_ms)
     achieved = flops_rank / (attend_avg * 1e-3) / 1e12
-    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    # The burst peak is cuBLAS timed alone; the sustained one a seconds-long loop
+    # under the power cap. A timed region shorter than that compares with burst.
+    region_s = ms_max * 1e-3
+    long_region = region_s >= SUSTAINED_REGION_S
+    peak = sustained if long_region else burst
+    peak_kind = (f"bf16 {'sustained' if long_region else 'burst'} ({peak_src}); timed region "
+                 f"{region_s:.3f} s")
+    per_clock = None
+    if clock_info and clock_info.get("sm_mhz"):
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        mhz = clock_info["sm_mhz"]
+        per_clock = {
+            "sm_mhz_median": mhz, "sms": sms,
+            "ms_x_mhz": attend_avg * mhz,
+            "flop_per_sm_clock": flops_rank / (attend_avg * 1e-3 * mhz * 1e6 * sms),
+            "dense_mma_flop_per_sm_clock": 8192,
+        }
     append_bytes = appends_per_chunk * 2 * 2 * (w.batch * w.chunk_len * w.heads * w.head_dim * 2)
     # (per append of one tier: K and V, each read once and written once)
     append_gbs = append_bytes / (statistics.fmean(append_ms) * 1e-3) / 1e9
@@ -634,7 +768,9 @@ def run_ours(args, w):
                 " (sparse, timed with its staging kernel)" if block_mask is not None else
                 " (frame-aligned, timed with its staging kernel)" if args.editing else ""),
             "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-            "peak_kind": f"bf16 sustained ({peak_src})", "frac_of_burst_peak": achieved / burst,
+            "peak_kind": peak_kind, "frac_of_burst_peak": achieved / burst,
+            "frac_of_sustained_peak": achieved / sustained,
+            "per_clock": per_clock,
             "traffic": kernel_traffic("attend_tc.cuh", w.name),
             "flops_per_launch": flops, "avg_launch_ms": attend_avg,
         },
@@ -655,6 +791,8 @@ def run_ours(args, w):
         "clocks": clock_info,
         "cpu_baseline": cpu,
     }
+    if gaps is not None:
+        line["launch_gaps"] = gaps
     print(json.dumps(line), flush=True)
     return 0
 

@@ -20,6 +20,7 @@ SA_ERR_STATE = 2
 SA_ERR_UNSUPPORTED = 3
 SA_ERR_CUDA = 4
 SA_ERR_TIMEOUT = 5
+SA_ERR_RANGE = 6
 SA_TIER_NOISY = 0
 SA_TIER_CLEAN = 1
 SA_MAX_ATTENDED = 16
@@ -80,7 +81,7 @@ _SIGNATURES = {
     "sa_debug_attend_stalled": (_I, [_P, _P, _P, _P, _I, _P, _P]),
     "sa_chunk_count": (_I, [_P, _I]),
     "sa_debug_inject_cuda_error": (_I, [_P]),
-    "sa_debug_layout": (_I, [_P, _I, _I32P, _I]),
+    "sa_debug_layout": (_I, [_P, _I, _I32P, _I32P, _I]),
     "sa_plan": (_I, [_CFGP, ctypes.c_int32, _I32P, _I32P, _I32P, _I]),
     "sa_stream_plan": (_I, [_P, _I, _I, _I32P, _I32P, _I32P, _I]),
     "sa_slot_of": (_I, [_CFGP, ctypes.c_int32]),
@@ -249,11 +250,12 @@ def sa_chunk_count(handle, tier):
 
 
 def sa_debug_layout(handle, tier, n):
-    buf = (ctypes.c_int32 * n)()
-    m = lib().sa_debug_layout(handle, tier, buf, n)
+    """(chunk id per slot, rank per slot) of one tier; -1 marks an empty slot."""
+    ids, ranks = (ctypes.c_int32 * n)(), (ctypes.c_int32 * n)()
+    m = lib().sa_debug_layout(handle, tier, ids, ranks, n)
     if m < 0:
         raise SaError(-m, last_error(handle))
-    return list(buf[:m])
+    return list(ids[:m]), list(ranks[:m])
 
 
 def sa_plan(cfg, chunk):

@@ -32,6 +32,11 @@ __global__ void __launch_bounds__(256) attend_simt_kernel(AttendParams p) {
   float qraw[DPL];
 #pragma unroll
   for (int d = 0; d < DPL; ++d) qraw[d] = __bfloat162float(qrow[lane * DPL + d]);
+  bool saturated = false;  // a pair above the fp16 maximum in norm (see rope.cuh)
+#pragma unroll
+  for (int d = 0; d < DPL; d += 2)
+    saturated |= fmaf(qraw[d], qraw[d], qraw[d + 1] * qraw[d + 1]) > kF16MaxSq;
+  if (saturated) atomicOr(p.status, kDevWarnSaturated);
 
   float m = -INFINITY, lsum = 0.f, acc[DPL];
 #pragma unroll

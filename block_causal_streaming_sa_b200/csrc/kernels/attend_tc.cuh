@@ -689,12 +689,15 @@ __global__ void __launch_bounds__(384, 1)
       {
         const uint4* src = reinterpret_cast<const uint4*>(p.q + row_off);
         const int td0 = groups[g0].t_delta;
+        bool saturated = false;
 #pragma unroll 2
         for (int c = 0; c < D / 8; ++c) {
           uint4 v = valid ? ld_nc_v4(src + c) : make_uint4(0u, 0u, 0u, 0u);
           if (c < T::kTChunks) st_shared_v4(q_raw + c * 16, v);
+          saturated |= pair_norm_exceeds_f16(v);
           st_shared_v4(q_smem + sw128_offset(r, c), rope_chunk(v, c, p.rope, td0 + f, y, x));
         }
+        if (saturated) atomicOr(p.status, kDevWarnSaturated);
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(bar(T::QREADY(i)));
       }

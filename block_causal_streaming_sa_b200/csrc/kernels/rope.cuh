@@ -41,6 +41,24 @@ __device__ __forceinline__ uint32_t rope_pair(uint32_t ab, float2 cs) {
   return ptx::pack_f16x2(fmaf(a, cs.x, -b * cs.y), fmaf(a, cs.y, b * cs.x));
 }
 
+// 65504^2 (exact in fp32): the squared largest finite fp16 value.
+constexpr float kF16MaxSq = 4290774016.0f;
+
+// True when one of the 4 bf16 pairs of a 16-byte chunk has a norm above 65504.
+// A rotation keeps each pair's norm, and at some angle one value of the pair
+// equals it, so such a pair saturates when rounded to fp16 for some position;
+// the test does not depend on the position, so relocation cannot change it.
+__device__ __forceinline__ bool pair_norm_exceeds_f16(uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float a = bf16_lo(w[i]), b = bf16_hi(w[i]);
+    m = fmaxf(m, fmaf(a, a, b * b));
+  }
+  return m > kF16MaxSq;
+}
+
 // Rotate the 8 bf16 values (4 pairs) of 16-byte chunk `c` of a head vector into
 // 8 fp16 values.
 __device__ __forceinline__ uint4 rope_chunk(uint4 v, int c, const RopeTables& rt, int pos_t, int y,
@@ -89,6 +107,7 @@ __global__ void rope_transpose_kernel(AppendParams p) {
   const int h = t / vec_per_head, c = t - h * vec_per_head;
   const int n_tok = p.B * p.L;
   const int tok0 = blockIdx.x * kRopeTokensPerBlock;
+  bool saturated = false;
   uint4 v[kRopeTokensPerBlock];
 #pragma unroll
   for (int k = 0; k < kRopeTokensPerBlock; ++k) {
@@ -104,10 +123,12 @@ __global__ void rope_transpose_kernel(AppendParams p) {
       const int f = l / p.rope.frame_tokens;
       const int y = (l / p.rope.tok_w) % p.rope.tok_h;
       const int x = l % p.rope.tok_w;
+      saturated |= pair_norm_exceeds_f16(v[k]);
       v[k] = rope_chunk(v[k], c, p.rope, f, y, x);
     }
     st_v4(out + ((static_cast<size_t>(b) * p.H + h) * p.L_out + l) * p.D + c * 8, v[k]);
   }
+  if (saturated) atomicOr(p.status, kDevWarnSaturated);
 }
 
 }  // namespace sa

@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -223,6 +224,30 @@ bool encode_blhd(CUtensorMap* map, const void* base, const Derived& d, int rows)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Memory type of a tensor pointer, queried on the host before anything is
+// launched: device memory (of `device`, or of any device when device < 0) or
+// managed memory passes; host memory (pageable or pinned) and unknown
+// addresses are refused. NULL passes (presence is checked by the callers).
+bool device_memory(const void* p, int device, const char* what, std::string* why) {
+  if (p == nullptr) return true;
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the sticky-free error of the failed query
+    *why = std::string(what) + " is not a CUDA pointer";
+    return false;
+  }
+  if (a.type == cudaMemoryTypeManaged) return true;
+  if (a.type != cudaMemoryTypeDevice) {
+    *why = std::string(what) + " is host memory; it must be device memory";
+    return false;
+  }
+  if (device >= 0 && a.device != device) {
+    *why = std::string(what) + " is on another device than the handle";
+    return false;
+  }
+  return true;
+}
+
 // Persistent grid: one CTA per SM at most; with the split tail allowed, a problem
 // of fewer work tiles than SMs gets two CTAs per tile (key-range halves).
 unsigned attend_grid(const Derived& d, int rows, int sm_count, bool split_ok) {
@@ -352,6 +377,16 @@ int check_device(sa_handle* h) {
   return SA_OK;
 }
 
+// Every non-NULL pointer must be device memory of the handle's device (or
+// managed memory); checked before anything is launched.
+int check_mem(sa_handle* h, std::initializer_list<std::pair<const void*, const char*>> ptrs) {
+  std::string why;
+  for (const auto& pr : ptrs)
+    if (!device_memory(pr.first, h->device, pr.second, &why))
+      return h->fail(SA_ERR_INVALID_ARG, why);
+  return SA_OK;
+}
+
 // Rotate K (and copy V, if given; rotate it too with second_is_key) of `rows`
 // tokens into [B, H, L_out, D] planes.
 int launch_rope_transpose(sa_handle* h, const void* K, const void* V, __nv_bfloat16* k_out,
@@ -370,6 +405,7 @@ int launch_rope_transpose(sa_handle* h, const void* K, const void* V, __nv_bfloa
   ap.L_out = L_out;
   ap.second_is_key = second_is_key ? 1 : 0;
   ap.rope = h->rope();
+  ap.status = h->status();
   const int threads = static_cast<int>(align_up(static_cast<size_t>(d.H) * d.D / 8, 32));
   const long long n_tok = 1LL * d.B * rows;
   dim3 grid(static_cast<unsigned>((n_tok + sa::kRopeTokensPerBlock - 1) / sa::kRopeTokensPerBlock),
@@ -492,7 +528,7 @@ int check_attend_ptrs(sa_handle* h, const void* Q, const void* Vc, const void* O
   if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
     return h->fail(SA_ERR_INVALID_ARG, "lse must be 4-byte aligned");
   if (O == Q || O == Vc) return h->fail(SA_ERR_INVALID_ARG, "O must not alias an input");
-  return SA_OK;
+  return check_mem(h, {{Q, "Q"}, {Vc, "Vc"}, {O, "O"}, {lse, "lse"}});
 }
 
 // Rotate the generating chunk's keys (and, for frame-aligned editing, its
@@ -507,6 +543,8 @@ int stage_keys(sa_handle* h, const void* Kc, int n_frames, sa_stream stream,
     return h->fail(SA_ERR_INVALID_ARG, "Kc must be a non-NULL 16-byte aligned pointer");
   if (Ks != nullptr && !aligned16(Ks))
     return h->fail(SA_ERR_INVALID_ARG, "Ks must be 16-byte aligned");
+  rc = check_mem(h, {{Kc, "Kc"}, {Ks, "Ks"}});
+  if (rc != SA_OK) return rc;
   if (h->count[0] != h->count[1])
     return h->fail(SA_ERR_STATE, "both tiers must hold the same chunks before attending");
   rc = check_device(h);
@@ -533,6 +571,8 @@ int attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final
   const bool aligned = Vs != nullptr;
   if (aligned && (!aligned16(Vs) || O == Vs))
     return h->fail(SA_ERR_INVALID_ARG, "Vs must be 16-byte aligned and not aliased by O");
+  rc = check_mem(h, {{Vs, "Vs"}, {block_mask, "block_mask"}});
+  if (rc != SA_OK) return rc;
   if (aligned && !h->staged_source)
     return h->fail(SA_ERR_STATE, "no source keys staged for frame-aligned attention");
   if (aligned && (simt || block_mask != nullptr))
@@ -612,6 +652,8 @@ int attend_common(sa_handle* h, const void* Q, const void* Kc, const void* Vc, i
   if (rc != SA_OK) return rc;
   if (block_mask != nullptr && h->has_ref)
     return h->fail(SA_ERR_UNSUPPORTED, "block-sparse attention takes no reference image");
+  rc = check_mem(h, {{Kc, "Kc"}, {block_mask, "block_mask"}});
+  if (rc != SA_OK) return rc;
   rc = stage_keys(h, Kc, n_frames, stream);
   if (rc != SA_OK) return rc;
   return attend_staged(h, Q, Vc, step_is_final, O, lse, stream, simt, false, block_mask);
@@ -634,6 +676,8 @@ int attend_aligned(sa_handle* h, const void* Q, const void* Kc, const void* Vc, 
   if (max_groups(h, true) > sa::kMaxGroups)
     return h->fail(SA_ERR_UNSUPPORTED, "more than SA_MAX_ATTENDED key groups (chunks, "
                                        "reference and source frames)");
+  rc = check_mem(h, {{Kc, "Kc"}, {Ks, "Ks"}, {Vs, "Vs"}});
+  if (rc != SA_OK) return rc;
   rc = stage_keys(h, Kc, n_frames, stream, Ks);
   if (rc != SA_OK) return rc;
   return attend_staged(h, Q, Vc, step_is_final, O, lse, stream, false, false, nullptr, Vs);
@@ -648,21 +692,61 @@ static __device__ __align__(256) uint8_t g_noalloc_keys[SA_NOALLOC_MAX_KEY_BYTES
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
-void* g_noalloc_addr[kMaxDevices] = {};
+// Per device ordinal: the array's address and the CUDA context it was looked up
+// in (a process-unique context id). A device reset or a new primary context
+// reloads the module, which may move the array, so a different context id
+// means the address is looked up again.
+struct NoallocAddr {
+  unsigned long long ctx_id;
+  void* ptr;
+};
+NoallocAddr g_noalloc_addr[kMaxDevices] = {};
+
+typedef CUresult (*PFN_ctx_get_current)(CUcontext*);
+typedef CUresult (*PFN_ctx_get_id)(CUcontext, unsigned long long*);
+
+// Id of the calling thread's current CUDA context (driver entry points found
+// through the runtime, so the library needs no link to libcuda).
+bool current_ctx_id(unsigned long long* id) {
+  static PFN_ctx_get_current get_current = nullptr;
+  static PFN_ctx_get_id get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_ctx_get_current>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_ctx_get_id>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS ||
+      ctx == nullptr)
+    return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 int noalloc_scratch(sa_handle* h, void** out) {
   if (h->device < 0 || h->device >= kMaxDevices)
     return h->fail(SA_ERR_UNSUPPORTED, "device ordinal too large for sa_attend_noalloc");
+  unsigned long long ctx = 0;
+  if (!current_ctx_id(&ctx))
+    return h->fail(SA_ERR_CUDA, "sa_attend_noalloc: no current CUDA context");
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_addr[h->device] == nullptr) {
+  NoallocAddr& a = g_noalloc_addr[h->device];
+  if (a.ptr == nullptr || a.ctx_id != ctx) {
     void* ptr = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_keys);
     if (e != cudaSuccess || ptr == nullptr)
       return h->fail(SA_ERR_CUDA, std::string("cudaGetSymbolAddress of the static key scratch: ") +
                                       cudaGetErrorString(e));
-    g_noalloc_addr[h->device] = ptr;
+    a.ptr = ptr;
+    a.ctx_id = ctx;
   }
-  *out = g_noalloc_addr[h->device];
+  *out = a.ptr;
   return SA_OK;
 }
 
@@ -673,6 +757,8 @@ int attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc, 
   if (Kc == nullptr || !aligned16(Kc) || O == Kc)
     return h->fail(SA_ERR_INVALID_ARG, "Kc must be non-NULL, 16-byte aligned, not aliased by O");
   rc = check_attend_ptrs(h, Q, Vc, O, lse);
+  if (rc != SA_OK) return rc;
+  rc = check_mem(h, {{Kc, "Kc"}});
   if (rc != SA_OK) return rc;
   if (h->count[0] != h->count[1])
     return h->fail(SA_ERR_STATE, "both tiers must hold the same chunks before attending");
@@ -724,6 +810,8 @@ int append_chunk(sa_handle* h, int tier, const void* K, const void* V, int n_fra
     return h->fail(SA_ERR_INVALID_ARG, "K and V must be 16-byte aligned");
   if (h->count[tier] > h->count[1 - tier])
     return h->fail(SA_ERR_STATE, "this tier is already one chunk ahead of the other");
+  rc = check_mem(h, {{K, "K"}, {V, "V"}});
+  if (rc != SA_OK) return rc;
   rc = check_device(h);
   if (rc != SA_OK) return rc;
   const Derived& d = h->d;
@@ -831,6 +919,9 @@ SA_API int sa_exchange_pack(const void* x, int B, int T, int C, int D, int G, in
     g_error = "exchange: x and buf must be non-NULL and 16-byte aligned";
     return SA_ERR_INVALID_ARG;
   }
+  if (!device_memory(x, -1, "exchange: x", &g_error) ||
+      !device_memory(buf, -1, "exchange: buf", &g_error))
+    return SA_ERR_INVALID_ARG;
   ep.x = static_cast<const __nv_bfloat16*>(x);
   ep.out = static_cast<uint8_t*>(buf);
   return launch_exchange(true, ep, stream);
@@ -849,11 +940,14 @@ SA_API int sa_exchange_pack_to(const void* x, int B, int T, int C, int D, int G,
     g_error = "exchange: x and dst_blocks must be non-NULL, x 16-byte aligned";
     return SA_ERR_INVALID_ARG;
   }
+  if (!device_memory(x, -1, "exchange: x", &g_error)) return SA_ERR_INVALID_ARG;
   for (int g = 0; g < G; ++g) {
     if (dst_blocks[g] == nullptr || !aligned16(dst_blocks[g])) {
       g_error = "exchange: every destination block must be non-NULL and 16-byte aligned";
       return SA_ERR_INVALID_ARG;
     }
+    if (!device_memory(dst_blocks[g], -1, "exchange: a destination block", &g_error))
+      return SA_ERR_INVALID_ARG;
     ep.dst[g] = static_cast<uint8_t*>(dst_blocks[g]);
   }
   ep.x = static_cast<const __nv_bfloat16*>(x);
@@ -936,6 +1030,9 @@ SA_API int sa_exchange_unpack(const void* buf, int B, int T, int C, int D, int G
     g_error = "exchange: buf and y must be non-NULL, 16-byte aligned and distinct";
     return SA_ERR_INVALID_ARG;
   }
+  if (!device_memory(buf, -1, "exchange: buf", &g_error) ||
+      !device_memory(y, -1, "exchange: y", &g_error))
+    return SA_ERR_INVALID_ARG;
   ep.in = static_cast<const uint8_t*>(buf);
   ep.y = static_cast<__nv_bfloat16*>(y);
   return launch_exchange(false, ep, stream);
@@ -1119,6 +1216,8 @@ SA_API int sa_set_reference(sa_handle* h, const void* K, const void* V, sa_strea
     return h->fail(SA_ERR_STATE, "the config has ref_frames == 0: no room for a reference image");
   if (K == nullptr || V == nullptr || !aligned16(K) || !aligned16(V))
     return h->fail(SA_ERR_INVALID_ARG, "K and V must both be non-NULL and 16-byte aligned");
+  rc = check_mem(h, {{K, "K"}, {V, "V"}});
+  if (rc != SA_OK) return rc;
   rc = check_device(h);
   if (rc != SA_OK) return rc;
   rc = launch_rope_transpose(h, K, V, h->ref(), h->ref() + h->d.ref_elems, h->d.Lref, h->d.Lref,
@@ -1239,17 +1338,27 @@ SA_API int sa_chunk_count(const sa_handle* h, int tier) {
   return h->count[tier];
 }
 
-SA_API int sa_debug_layout(const sa_handle* h, int tier, int32_t* slot_chunk_ids, int n) {
+SA_API int sa_debug_layout(const sa_handle* h, int tier, int32_t* slot_chunk_ids,
+                           int32_t* slot_ranks, int n) {
   if (h == nullptr || slot_chunk_ids == nullptr || (tier != SA_TIER_NOISY && tier != SA_TIER_CLEAN))
     return -SA_ERR_INVALID_ARG;
   const Derived& d = h->d;
   const int slots = d.S + d.R;
   const int m = n < slots ? n : slots;
-  for (int s = 0; s < m; ++s) slot_chunk_ids[s] = -1;
+  int held[SA_MAX_ATTENDED];
+  for (int s = 0; s < slots; ++s) held[s] = -1;
   const int cnt = h->count[tier];
   for (int j = 0; j < cnt; ++j) {  // the latest chunk written to a slot holds it
     const int s = slot_of(d, j);
-    if (s >= 0 && s < m) slot_chunk_ids[s] = j;
+    if (s >= 0) held[s] = j;
+  }
+  for (int s = 0; s < m; ++s) {
+    slot_chunk_ids[s] = held[s];
+    if (slot_ranks == nullptr) continue;
+    // rank = number of held chunks older than this one (ascending id order)
+    int rank = 0;
+    for (int u = 0; u < slots; ++u) rank += held[u] >= 0 && held[u] < held[s];
+    slot_ranks[s] = held[s] < 0 ? -1 : rank;
   }
   return m;
 }
@@ -1320,6 +1429,10 @@ SA_API int sa_get_status(sa_handle* h, sa_stream stream) {
     return h->fail(SA_ERR_CUDA, std::string("reading the status word: ") +
                                     cudaGetErrorString(cudaGetLastError()));
   if (word & sa::kDevErrTimeout) return h->fail(SA_ERR_TIMEOUT, "a kernel gave up a bounded wait");
+  if (word & sa::kDevWarnSaturated)
+    return h->fail(SA_ERR_RANGE,
+                   "a Q or K pair had a norm above 65504 and was saturated to fp16 for the "
+                   "score MMA");
   return SA_OK;
 }
 
@@ -1335,6 +1448,7 @@ SA_API const char* sa_status_string(int status) {
     case SA_ERR_UNSUPPORTED: return "SA_ERR_UNSUPPORTED";
     case SA_ERR_CUDA: return "SA_ERR_CUDA";
     case SA_ERR_TIMEOUT: return "SA_ERR_TIMEOUT";
+    case SA_ERR_RANGE: return "SA_ERR_RANGE";
     default: return "SA_ERR_UNKNOWN";
   }
 }

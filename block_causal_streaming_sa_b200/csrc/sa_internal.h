@@ -19,8 +19,11 @@ constexpr int kModeDense = 0;
 constexpr int kModeSparse = 1;
 constexpr int kModeAligned = 2;
 
-// Device status word bits (written with atomicOr, read by sa_get_status).
+// Device status word bits (written with atomicOr, read by sa_get_status):
+// a bounded wait ran out; a Q or K pair had a norm above the fp16 maximum, so
+// its rotated values were saturated for the score MMA.
 constexpr unsigned kDevErrTimeout = 1u;
+constexpr unsigned kDevWarnSaturated = 2u;
 
 // fp32 (cos, sin) tables of the three RoPE bands (reading: bands [t | h | w] of
 // D - 4*(D/6), 2*(D/6), 2*(D/6) dims, pair i of a band of size d turned by
@@ -47,6 +50,7 @@ struct AppendParams {
   int L_out;  // rows per output plane
   int second_is_key;
   RopeTables rope;
+  unsigned* status;  // device status word (kDevWarnSaturated)
 };
 
 // One attended key group: the reference image first (if set), then the

@@ -166,6 +166,11 @@ class StreamingAttention:
         return B.sa_chunk_count(self.handle, tier)
 
     def layout(self, tier):
+        """Chunk id held by each slot of the tier (-1: empty)."""
+        return self.layout_ranks(tier)[0]
+
+    def layout_ranks(self, tier):
+        """(chunk id per slot, rank of that chunk in the next attention's list)."""
         c = self.cfg_dict
         return B.sa_debug_layout(self.handle, tier, c["sink_chunks"] + c["window_chunks"] - 1)
 

@@ -38,6 +38,10 @@
  *    passed as sa_stream; NULL is the legacy default stream). After sa_create,
  *    the append, reference, staging and attention calls allocate no memory and
  *    never synchronise the host (sa_reset and sa_get_status do synchronise).
+ *  - Before anything is launched, every tensor pointer is checked on the host
+ *    (cudaPointerGetAttributes): it must be device memory of the handle's
+ *    device or managed memory, else SA_ERR_INVALID_ARG. A host pointer
+ *    (pageable or pinned) is refused, not read by a kernel.
  *  - The device calls can be captured into a CUDA graph. A captured attention
  *    keeps the plan of the chunk it was captured for (attended chunks, slots
  *    and relocated positions are launch arguments): replay it for that chunk's
@@ -67,7 +71,9 @@ typedef enum {
   SA_ERR_STATE = 2,        /* call not allowed in the handle's current state */
   SA_ERR_UNSUPPORTED = 3,  /* valid request the library does not serve (e.g. D) */
   SA_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed */
-  SA_ERR_TIMEOUT = 5       /* a kernel gave up a bounded wait (device status) */
+  SA_ERR_TIMEOUT = 5,      /* a kernel gave up a bounded wait (device status) */
+  SA_ERR_RANGE = 6         /* an operand left the fp16 range of the score MMA and
+                              was saturated (device status; outputs degraded) */
 } sa_status;
 
 typedef enum { SA_TIER_NOISY = 0, SA_TIER_CLEAN = 1 } sa_tier;
@@ -126,8 +132,12 @@ SA_API int sa_reset(sa_handle* h);
  * window slot S + (n - S) mod (W - 1), overwriting (evicting) the oldest
  * non-sink chunk once the window is full; with W == 1 a non-sink chunk is not
  * stored. K is rotated by its in-chunk (frame, row, column) position on the way
- * in and kept as fp16 (the score MMA's operand type; rotated pairs must keep a
- * norm below 65504, larger ones saturate); V is kept as bf16. The relocated
+ * in and kept as fp16 (the score MMA's operand type). A pair (2i, 2i+1) whose
+ * norm exceeds 65504, the fp16 maximum, is out of range: at some rotation
+ * angles its values leave fp16 and are saturated to +-65504. The device status
+ * word records every such pair whatever its angle (sa_get_status then returns
+ * SA_ERR_RANGE until sa_reset); the same check covers Q and the keys of every
+ * other call. V is kept as bf16. The relocated
  * temporal offset is applied at attend time.
  * A tier may run at most one chunk ahead of the other: appending to the tier
  * that is already ahead is SA_ERR_STATE. K and V may be freed once the launch
@@ -263,6 +273,9 @@ SA_API int sa_attend_staged(sa_handle* h, const void* Q, const void* Vc, int ste
  *    handles) race; order them (one stream, or events);
  *  - the first call on a device looks up the array's device address (a
  *    runtime symbol query); make that first call before any stream capture.
+ *    The address is kept per device together with the CUDA context it was
+ *    found in: after a device reset (cudaDeviceReset) or in a new context the
+ *    first call looks it up again, so make that call, too, outside capture.
  * Returns the same statuses as sa_attend. */
 #define SA_NOALLOC_MAX_KEY_BYTES (64u << 20)
 SA_API int sa_attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc,
@@ -298,9 +311,18 @@ SA_API int sa_debug_inject_cuda_error(sa_handle* h);
 /* Chunks appended so far to `tier`, or a negative sa_status. */
 SA_API int sa_chunk_count(const sa_handle* h, int tier);
 
-/* Chunk id held by each slot of `tier` (-1 = empty), for the first
- * min(n, S + W - 1) slots; returns the number of slots written. Host only. */
-SA_API int sa_debug_layout(const sa_handle* h, int tier, int32_t* slot_chunk_ids, int n);
+/* Cache layout of `tier`, for bit-exact checks of the ring and the relocation
+ * ("Vidu S2 vs PixVerse R2", section 选择三：有上限的记忆: sinks kept, the window
+ * slides, positions relocated). For each of the first min(n, S + W - 1) slots:
+ * slot_chunk_ids[s] = the chunk id the slot holds (-1 = empty), and, if
+ * slot_ranks is not NULL, slot_ranks[s] = the rank of that chunk among the
+ * chunks the next attention of this tier reads (the held chunks in ascending
+ * id order, then the generating chunk; -1 = empty slot). The chunk's temporal
+ * base is ref_frames + rank * F when every chunk has F frames (sa_stream_plan
+ * gives the bases for chunks of any length). Returns the number of slots
+ * written, or a negative sa_status. Host only. */
+SA_API int sa_debug_layout(const sa_handle* h, int tier, int32_t* slot_chunk_ids,
+                           int32_t* slot_ranks, int n);
 
 /* The attention plan of chunk `chunk` of a stream with config cfg whose chunks
  * all have F frames, computed on the host with no handle and no device: writes,
@@ -384,8 +406,11 @@ SA_API int sa_ipc_close(void* dev_ptr);
 /* Slot of chunk id `chunk` in a tier (-1 if it is never stored). Host only. */
 SA_API int sa_slot_of(const sa_config* cfg, int32_t chunk);
 
-/* Wait for `stream`, then read and return the device status word: SA_OK, or
- * SA_ERR_TIMEOUT if a kernel gave up a bounded wait since the last reset. */
+/* Wait for `stream`, then read and return the device status word: SA_OK;
+ * SA_ERR_TIMEOUT if a kernel gave up a bounded wait since the last reset;
+ * else SA_ERR_RANGE if a rotated Q or K pair of some call since the last reset
+ * had a norm above 65504 and was saturated to fp16 (the outputs were computed
+ * with the saturated values). */
 SA_API int sa_get_status(sa_handle* h, sa_stream stream);
 
 /* Text of the handle's last error (never NULL); with h == NULL, of the last

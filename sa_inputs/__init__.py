@@ -75,6 +75,14 @@ def normals(seed, count):
     return out
 
 
+def _uniform_at(seed, pos):
+    """Draw ``pos`` (int64 array of stream positions) of stream ``seed``, as
+    ``uniforms`` would give it."""
+    with np.errstate(over="ignore"):
+        z = _mix(np.uint64(seed) + (pos.astype(np.uint64) + np.uint64(1)) * _GAMMA)
+    return (z >> np.uint64(11)).astype(np.float64) * (1.0 / (1 << 53))
+
+
 def seed_of(*fields):
     """Stable 64-bit seed of a tuple of names and numbers."""
     key = "|".join(str(f) for f in fields).encode()
@@ -99,6 +107,22 @@ def normal_bf16(seed, shape, scale=1.0, outlier_frac=0.0, outlier_mag=8.0):
 
     _blocks(count, fill)
     return torch.from_numpy(out.reshape(shape)).to(torch.bfloat16)
+
+
+def normal_bf16_at(seed, index, scale=1.0, outlier_frac=0.0, outlier_mag=8.0):
+    """The elements at flat C-order positions ``index`` (int64 array, any shape)
+    of ``normal_bf16(seed, shape, ...)``, as a bf16 CPU tensor of index's shape:
+    the generator is counter-based, so element i depends only on (seed, i) and a
+    slice of a large tensor can be drawn without drawing the rest."""
+    i = np.asarray(index, dtype=np.int64).reshape(-1)
+    u1, u2 = _uniform_at(seed, 2 * i), _uniform_at(seed, 2 * i + 1)
+    v = np.sqrt(-2.0 * np.log1p(-u1)) * np.cos(2.0 * np.pi * u2) * scale
+    if outlier_frac > 0.0:
+        pick = _uniform_at(seed_of(seed, "outlier"), i) < outlier_frac
+        sign = np.where(_uniform_at(seed_of(seed, "sign"), i) < 0.5, -1.0, 1.0)
+        v = np.where(pick, sign * outlier_mag, v)
+    out = v.astype(np.float32).reshape(np.shape(index))
+    return torch.from_numpy(out).to(torch.bfloat16)
 
 
 def device_normal_bf16(seed, shape, device):
@@ -155,6 +179,18 @@ class Workload:
         return normal_bf16(seed_of(self.name, layer, chunk, step, name), self.shape(),
                            scale=scale, outlier_frac=self.outlier_frac,
                            outlier_mag=self.outlier_mag)
+
+    def tensor_at(self, name, chunk, step=0, layer=0, batches=None, heads=None):
+        """The (batch, head) slices ``tensor(...)[batches][:, :, heads]`` of a
+        seeded tensor, [nb, L, nh, D], drawn without drawing the whole tensor."""
+        b = np.arange(self.batch) if batches is None else np.asarray(batches)
+        h = np.arange(self.heads) if heads is None else np.asarray(heads)
+        L, H, D = self.chunk_len, self.heads, self.head_dim
+        idx = (((b[:, None, None, None] * L + np.arange(L)[None, :, None, None]) * H
+                + h[None, None, :, None]) * D + np.arange(D)[None, None, None, :])
+        scale = self.k_scale if name.startswith("K") else 1.0
+        return normal_bf16_at(seed_of(self.name, layer, chunk, step, name), idx, scale=scale,
+                              outlier_frac=self.outlier_frac, outlier_mag=self.outlier_mag)
 
     def config_dict(self):
         return dict(batch=self.batch, heads=self.heads, head_dim=self.head_dim,

@@ -112,8 +112,13 @@ class Pair:
         return o_gpu, o_ref, l_gpu, l_ref
 
     def check_layout(self):
+        """Slot contents and relocated ranks of both tiers, bit-exact."""
         for tier in (NOISY, CLEAN):
-            got = self.gpu.layout(tier)
-            want = [-1 if s is None else s for s in self.oracle.model[tier].slots]
+            got, got_ranks = self.gpu.layout_ranks(tier)
+            model = self.oracle.model[tier]
+            want = [-1 if s is None else s for s in model.slots]
             assert got == want, (tier, got, want)
-            assert self.gpu.chunk_count(tier) == self.oracle.model[tier].count
+            ranks = model.ranks()
+            want_ranks = [-1 if s is None else ranks[s] for s in model.slots]
+            assert got_ranks == want_ranks, (tier, got_ranks, want_ranks)
+            assert self.gpu.chunk_count(tier) == model.count

@@ -175,3 +175,30 @@ def test_exchange_block_bytes_and_shape_checks():
         assert sa.sa_exchange_block_bytes(*bad) == 0, bad
     with pytest.raises(sa.SaError):
         sa.sa_exchange_pack(0, 1, 8, 4, 64, 2, 1, P8, 0)
+
+
+def test_status_codes_match_the_header():
+    """The binding's status constants are the header's enum values, and every
+    one has a name."""
+    import re
+
+    text = open(sa._binding.HEADER).read()
+    enum = text[text.index("typedef enum {"):text.index("} sa_status;")]
+    codes = {m.group(1): int(m.group(2)) for m in re.finditer(r"(SA_\w+)\s*=\s*(\d+)", enum)}
+    assert codes == {n: getattr(sa._binding, n) for n in codes}
+    assert set(codes) >= {"SA_OK", "SA_ERR_TIMEOUT", "SA_ERR_RANGE"}
+    for name, value in codes.items():
+        assert sa._binding.status_name(value) == name
+
+
+def test_debug_layout_and_host_pointers_without_a_gpu():
+    lib = sa.lib()
+    ids = (ctypes.c_int32 * 4)()
+    assert lib.sa_debug_layout(None, 0, ids, None, 4) < 0
+    # exchange: a host pointer is not device memory (no GPU here: not a CUDA pointer)
+    x = torch.zeros((1, 8, 4, 64), dtype=torch.bfloat16)
+    buf = torch.zeros(1 << 14, dtype=torch.uint8)
+    with pytest.raises(sa.SaError) as e:
+        sa.sa_exchange_pack(x.data_ptr(), 1, 8, 4, 64, 2, 1, sa.SA_PAYLOAD_FP8, buf.data_ptr())
+    assert e.value.status == sa.SA_ERR_INVALID_ARG
+    assert "exchange: x" in sa.last_error()

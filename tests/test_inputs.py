@@ -40,3 +40,17 @@ def test_workload_shapes():
     t = WORKLOADS["tiny"].tensor("Q", chunk=0)
     assert tuple(t.shape) == (1, 192, 2, 64)
     assert torch.equal(t, WORKLOADS["tiny"].tensor("Q", chunk=0))
+
+
+def test_tensor_slices_equal_the_whole_tensor():
+    """tensor_at draws exactly the (batch, head) slices of the full tensor,
+    outliers and the K scale included (the generator is counter-based)."""
+    from sa_inputs import Workload
+
+    w = Workload("slices", 3, 5, 64, 2, 6, 7, sink=1, window=2, steps=1, stream=2,
+                 k_scale=0.5, outlier_frac=0.02)
+    for name in ("Q", "Kn"):
+        full = w.tensor(name, 4, 1, 2)
+        part = w.tensor_at(name, 4, 1, 2, batches=[0, 2], heads=[1, 4])
+        assert torch.equal(part, full[[0, 2]][:, :, [1, 4]])
+    assert torch.equal(w.tensor_at("Vc", 0), w.tensor("Vc", 0))
