@@ -8,7 +8,7 @@ PyTorch) and passes tensors' device pointers and the current CUDA stream.
 
 from ._binding import (  # noqa: F401
     SA_OK, SA_ERR_INVALID_ARG, SA_ERR_STATE, SA_ERR_UNSUPPORTED, SA_ERR_CUDA, SA_ERR_TIMEOUT,
-    SA_ERR_RANGE,
+    SA_ERR_RANGE, SA_ERR_BOUNDS, SA_BUILD_DEVICE_CHECKS, sa_build_info,
     SA_TIER_NOISY, SA_TIER_CLEAN, SaConfig, SaError, make_config, lib, header_symbols,
     sa_validate_config, sa_required_bytes, sa_create, sa_destroy, sa_reset, sa_append_chunk,
     sa_append_chunk_frames, sa_set_reference, sa_attend, sa_attend_frames, sa_attend_aligned,

@@ -11,7 +11,10 @@ import os
 import re
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libsa.so")
+# SA_LIBRARY=checked selects the checked build (device-side bounds checks,
+# include/sa.h: sa_build_info); the default is the release build.
+LIB_PATH = os.path.join(HERE, "libsa_checked.so" if os.environ.get("SA_LIBRARY") == "checked"
+                        else "libsa.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "sa.h")
 
 SA_OK = 0
@@ -21,6 +24,8 @@ SA_ERR_UNSUPPORTED = 3
 SA_ERR_CUDA = 4
 SA_ERR_TIMEOUT = 5
 SA_ERR_RANGE = 6
+SA_ERR_BOUNDS = 7
+SA_BUILD_DEVICE_CHECKS = 1
 SA_TIER_NOISY = 0
 SA_TIER_CLEAN = 1
 SA_MAX_ATTENDED = 16
@@ -97,6 +102,7 @@ _SIGNATURES = {
     "sa_get_status": (_I, [_P, _P]),
     "sa_last_error": (ctypes.c_char_p, [_P]),
     "sa_status_string": (ctypes.c_char_p, [_I]),
+    "sa_build_info": (_I, []),
 }
 
 
@@ -285,6 +291,11 @@ def sa_slot_of(cfg, chunk):
 
 def sa_get_status(handle, stream=0):
     return lib().sa_get_status(handle, _P(stream))
+
+
+def sa_build_info():
+    """Build flags of the loaded library (SA_BUILD_DEVICE_CHECKS: the checked build)."""
+    return lib().sa_build_info()
 
 
 def sa_exchange_block_bytes(B, T, C, D, G, split_dim, payload=SA_PAYLOAD_FP8):

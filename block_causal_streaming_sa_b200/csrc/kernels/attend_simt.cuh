@@ -28,7 +28,10 @@ __global__ void __launch_bounds__(256) attend_simt_kernel(AttendParams p) {
   const int y = (l / p.rope.tok_w) % p.rope.tok_h;
   const int x = l % p.rope.tok_w;
 
-  const __nv_bfloat16* qrow = p.q + ((static_cast<size_t>(b) * p.L + l) * p.H + h) * D;
+  const size_t row_off = ((static_cast<size_t>(b) * p.L + l) * p.H + h) * D;
+  const __nv_bfloat16* qrow = p.q + row_off;
+  // checked build: the row of Q and O lies inside the tensors
+  if (!SA_IN_BOUNDS(p.status, row_off + D, p.q_elems)) return;
   float qraw[DPL];
 #pragma unroll
   for (int d = 0; d < DPL; ++d) qraw[d] = __bfloat162float(qrow[lane * DPL + d]);
@@ -56,6 +59,11 @@ __global__ void __launch_bounds__(256) attend_simt_kernel(AttendParams p) {
     }
     const __nv_bfloat16 *kb, *vb;
     size_t vstride;
+#ifdef SA_DEVICE_CHECKS
+    const __nv_bfloat16* k_lo;  // the buffer the group's keys and values lie in
+    unsigned long long k_size, v_size;
+    const __nv_bfloat16* v_lo;
+#endif
     if (grp.src == 0) {
       kb = p.cache + ((static_cast<size_t>(grp.slot) * 2 * p.B + b) * p.H + h) * plane;
       vb = p.cache + (((static_cast<size_t>(grp.slot) * 2 + 1) * p.B + b) * p.H + h) * plane;
@@ -69,6 +77,25 @@ __global__ void __launch_bounds__(256) attend_simt_kernel(AttendParams p) {
       vb = p.v_cur + static_cast<size_t>(b) * p.L * p.H * D + static_cast<size_t>(h) * D;
       vstride = static_cast<size_t>(p.H) * D;
     }
+#ifdef SA_DEVICE_CHECKS
+    if (grp.src == 0) {
+      k_lo = v_lo = p.cache;
+      k_size = v_size = p.cache_elems;
+    } else if (grp.src == 2) {
+      k_lo = v_lo = p.ref;
+      k_size = v_size = p.ref_elems;
+    } else {
+      k_lo = p.k_cur;
+      k_size = p.kcur_elems;
+      v_lo = p.v_cur;
+      v_size = p.q_elems;
+    }
+    const unsigned long long k_end = static_cast<unsigned long long>(kb - k_lo) +
+                                     static_cast<unsigned long long>(grp.len - 1) * D + D;
+    const unsigned long long v_end = static_cast<unsigned long long>(vb - v_lo) +
+                                     static_cast<unsigned long long>(grp.len - 1) * vstride + D;
+    if (!SA_IN_BOUNDS(p.status, k_end, k_size) || !SA_IN_BOUNDS(p.status, v_end, v_size)) continue;
+#endif
     for (int n = 0; n < grp.len; ++n) {
       const __nv_bfloat16* kr = kb + static_cast<size_t>(n) * D + lane * DPL;
       const __nv_bfloat16* vr = vb + static_cast<size_t>(n) * vstride + lane * DPL;
@@ -92,8 +119,9 @@ __global__ void __launch_bounds__(256) attend_simt_kernel(AttendParams p) {
   const float inv = 1.f / lsum;
 #pragma unroll
   for (int d = 0; d < DPL; ++d) orow[lane * DPL + d] = __float2bfloat16_rn(acc[d] * inv);
-  if (p.lse != nullptr && lane == 0)
-    p.lse[(static_cast<size_t>(b) * p.H + h) * p.L + l] = (m + log2f(lsum)) * 0.69314718055994531f;
+  const size_t lse_idx = (static_cast<size_t>(b) * p.H + h) * p.L + l;
+  if (p.lse != nullptr && lane == 0 && SA_IN_BOUNDS(p.status, lse_idx + 1, p.lse_elems))
+    p.lse[lse_idx] = (m + log2f(lsum)) * 0.69314718055994531f;
 }
 
 }  // namespace sa

@@ -145,6 +145,11 @@ __device__ __noinline__ void epilogue(const AttendParams& p, uint32_t tO, bool a
   const float inv = seen ? 1.f / lsum : 0.f;
   const float lse_own = seen ? (m + __log2f(lsum)) * 0.69314718055994531f : -INFINITY;
   uint4* dst = reinterpret_cast<uint4*>(p.o + row_off);
+  // checked build: the row of O and the lse entry lie inside their buffers
+  valid = valid && SA_IN_BOUNDS(p.status, row_off + D, p.q_elems);
+  const bool lse_ok =
+      p.lse != nullptr && SA_IN_BOUNDS(p.status, static_cast<unsigned long long>(lse_idx) + 1,
+                                       p.lse_elems);
   if (half < 0) {
 #pragma unroll 1
     for (int j = 0; j < D / 32; ++j) {
@@ -171,11 +176,12 @@ __device__ __noinline__ void epilogue(const AttendParams& p, uint32_t tO, bool a
         }
       }
     }
-    if (valid && p.lse != nullptr) p.lse[lse_idx] = lse_own;
+    if (valid && lse_ok) p.lse[lse_idx] = lse_own;
     return;
   }
   const size_t prow = ((static_cast<size_t>(slot) * 2 + i) * 2 + half) * T::BM + r;
   const size_t qrow = ((static_cast<size_t>(slot) * 2 + i) * 2 + (1 - half)) * T::BM + r;
+  if (!SA_IN_BOUNDS(p.status, (prow > qrow ? prow : qrow) + 1, p.split_rows)) return;
   float* po = p.split_o + prow * D;
 #pragma unroll 1
   for (int j = 0; j < D / 32; ++j) {
@@ -223,7 +229,7 @@ __device__ __noinline__ void epilogue(const AttendParams& p, uint32_t tO, bool a
       q4.w = ptx::pack_bf16x2(fmaf(w1, b1.z, w0 * a1.z), fmaf(w1, b1.w, w0 * a1.w));
       st_v4(dst + c / 8, q4);
     }
-    if (p.lse != nullptr) p.lse[lse_idx] = lse_tot;
+    if (lse_ok) p.lse[lse_idx] = lse_tot;
   }
   *sem = 0;  // ready for the next launch
 }
@@ -357,6 +363,10 @@ __global__ void __launch_bounds__(384, 1)
   auto next_set = [&](const unsigned long long* row, int from, int hi) -> int {
     if (row == nullptr || from >= hi) return hi;
     int wd = from >> 6;
+#ifdef SA_DEVICE_CHECKS
+    const unsigned long long row0 = static_cast<unsigned long long>(row - p.block_bits);
+    if (!SA_IN_BOUNDS(p.status, row0 + n_words, p.bits_words)) return hi;
+#endif
     unsigned long long bits = __ldg(row + wd) & (~0ull << (from & 63));
     while (bits == 0ull) {
       if (++wd << 6 >= hi) return hi;
@@ -692,7 +702,9 @@ __global__ void __launch_bounds__(384, 1)
         bool saturated = false;
 #pragma unroll 2
         for (int c = 0; c < D / 8; ++c) {
-          uint4 v = valid ? ld_nc_v4(src + c) : make_uint4(0u, 0u, 0u, 0u);
+          uint4 v = valid && SA_IN_BOUNDS(p.status, row_off + c * 8 + 8, p.q_elems)
+                        ? ld_nc_v4(src + c)
+                        : make_uint4(0u, 0u, 0u, 0u);
           if (c < T::kTChunks) st_shared_v4(q_raw + c * 16, v);
           saturated |= pair_norm_exceeds_f16(v);
           st_shared_v4(q_smem + sw128_offset(r, c), rope_chunk(v, c, p.rope, td0 + f, y, x));

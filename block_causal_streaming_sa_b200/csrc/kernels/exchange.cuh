@@ -27,6 +27,7 @@
 
 #include "../sa_internal.h"
 #include "ptx.cuh"
+#include "rope.cuh"
 
 namespace sa {
 
@@ -80,164 +81,160 @@ __device__ __forceinline__ float2 e4m3x2_to_f32(uint16_t v) {
   return f;
 }
 
-// Vectors per warp: each lane issues the loads of all of them before the first
-// store, so enough bytes are in flight to cover memory latency.
-constexpr int kExchangeVecPerWarp = 4;
-
-// One warp per kExchangeVecPerWarp consecutive vectors of x; lane l holds
-// elements l*E .. l*E + E - 1 of each (E = D / 32).
+// Lanes per (b, t, c) vector: each lane moves 8 elements (16 bytes of bf16), so
+// a warp holds 32 / kLanes<D> vectors at a time; every lane issues the loads of
+// kExchangeSteps such groups before its first store, so enough bytes are in
+// flight to cover memory latency.
 template <int D>
-__global__ void __launch_bounds__(256) exchange_pack_kernel(ExchangeParams p) {
-  constexpr int E = D / 32, V = kExchangeVecPerWarp;
-  const long long vec0 = (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * V;
-  const int lane = threadIdx.x & 31;
-  const long long n_vec = static_cast<long long>(p.B) * p.T * p.C;
-  // E bf16 values of this lane as E / 2 packed 32-bit words, for each vector
-  uint32_t w[V][E / 2];
-#pragma unroll
-  for (int k = 0; k < V; ++k) {
-    if (vec0 + k >= n_vec) break;
-    const __nv_bfloat16* src = p.x + (vec0 + k) * D + lane * E;
-    if constexpr (E == 4) {
-      const uint2 u = *reinterpret_cast<const uint2*>(src);
-      w[k][0] = u.x;
-      w[k][1] = u.y;
-    } else {
-      w[k][0] = *reinterpret_cast<const uint32_t*>(src);
+constexpr int kLanes = D / 8;
+constexpr int kExchangeSteps = 4;
+template <int D>
+constexpr int kExchangeVecPerWarp = (32 / kLanes<D>) * kExchangeSteps;
+
+// Advance a (b, t, c) position over [B][T][C] by `step` vectors (step >= 1).
+__device__ __forceinline__ void exchange_step(int step, int C, int T, int& b, int& t, int& c) {
+  c += step;
+  while (c >= C) {
+    c -= C;
+    if (++t == T) {
+      t = 0;
+      ++b;
     }
   }
-  // (b, t, c) of the first vector once (64-bit division is a long routine),
-  // then stepped for the next ones
+}
+
+// kLanes<D> lanes per vector of x: the amax of a vector is reduced over its lanes
+// by shuffles; lane 0 of the vector writes its scale.
+template <int D>
+__global__ void __launch_bounds__(256) exchange_pack_kernel(ExchangeParams p) {
+  constexpr int LPV = kLanes<D>, VPW = 32 / LPV, S = kExchangeSteps;
+  const int lane = threadIdx.x & 31, sub = lane / LPV, sl = lane - sub * LPV;
+  const long long n_vec = static_cast<long long>(p.B) * p.T * p.C;
+  const long long base =
+      (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * kExchangeVecPerWarp<D>;
+  uint4 w[S];
+#pragma unroll
+  for (int s = 0; s < S; ++s) {
+    const long long vec = base + s * VPW + sub;
+    w[s] = vec < n_vec ? ld_nc_v4(p.x + vec * D + sl * 8) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  // (b, t, c) of this lane's first vector once (64-bit division is a long
+  // routine), then stepped
   int c = 0, t = 0, b = 0;
-  if (vec0 < n_vec) {
-    c = static_cast<int>(vec0 % p.C);
-    const long long bt = vec0 / p.C;
+  if (base + sub < n_vec) {
+    const long long vec = base + sub;
+    c = static_cast<int>(vec % p.C);
+    const long long bt = vec / p.C;
     t = static_cast<int>(bt % p.T);
     b = static_cast<int>(bt / p.T);
   }
 #pragma unroll
-  for (int k = 0; k < V; ++k) {
-    const long long vec = vec0 + k;
-    if (vec >= n_vec) break;
-    if (k > 0 && ++c == p.C) {
-      c = 0;
-      if (++t == p.T) {
-        t = 0;
-        ++b;
-      }
-    }
-    int g;
-    long long v;
-    exchange_place(p, b, t, c, g, v);
+  for (int s = 0; s < S; ++s) {
+    if (s > 0) exchange_step(VPW, p.C, p.T, b, t, c);
+    const bool active = base + s * VPW + sub < n_vec;
+    int g = 0;
+    long long v = 0;
+    if (active) exchange_place(p, b, t, c, g, v);
     uint8_t* blk = p.out != nullptr ? p.out + g * p.block_bytes : p.dst[g];
     if (!p.fp8) {
-      uint32_t* dst = reinterpret_cast<uint32_t*>(reinterpret_cast<__nv_bfloat16*>(blk) + v * D +
-                                                  lane * E);
-#pragma unroll
-      for (int i = 0; i < E / 2; ++i) dst[i] = w[k][i];
+      if (active) st_v4(reinterpret_cast<__nv_bfloat16*>(blk) + v * D + sl * 8, w[s]);
       continue;
     }
-    float f[E];
+    const uint32_t ww[4] = {w[s].x, w[s].y, w[s].z, w[s].w};
+    float f[8];
 #pragma unroll
-    for (int i = 0; i < E / 2; ++i) {
-      f[2 * i] = __uint_as_float(w[k][i] << 16);
-      f[2 * i + 1] = __uint_as_float(w[k][i] & 0xFFFF0000u);
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(ww[i] << 16);
+      f[2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u);
     }
-    float amax = 0.f;
+    float amax = fmaxf(fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3]))),
+                       fmaxf(fmaxf(fabsf(f[4]), fabsf(f[5])), fmaxf(fabsf(f[6]), fabsf(f[7]))));
+    // every lane takes part (inactive ones with zeros): the shuffles need the full warp
 #pragma unroll
-    for (int i = 0; i < E; ++i) amax = fmaxf(amax, fabsf(f[i]));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
+    for (int off = LPV / 2; off > 0; off >>= 1)
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     const float scale = __fdiv_rn(amax, kE4m3Max);
     const float inv = amax > 0.f ? __fdiv_rn(kE4m3Max, amax) : 0.f;
-    uint8_t* codes = blk + v * D + lane * E;
-    uint16_t q[E / 2];
-#pragma unroll
-    for (int i = 0; i < E / 2; ++i)
-      q[i] = scale > 0.f ? e4m3x2(__fmul_rn(f[2 * i], inv), __fmul_rn(f[2 * i + 1], inv))
-                         : static_cast<uint16_t>(0);
-    if constexpr (E == 4)
-      *reinterpret_cast<uint32_t*>(codes) = static_cast<uint32_t>(q[0]) |
-                                            (static_cast<uint32_t>(q[E / 2 - 1]) << 16);
-    else
-      *reinterpret_cast<uint16_t*>(codes) = q[0];
-    if (lane == 0) reinterpret_cast<float*>(blk + p.scale_off)[v] = scale;
+    uint2 q = make_uint2(0u, 0u);
+    if (scale > 0.f) {
+      q.x = static_cast<uint32_t>(e4m3x2(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv))) |
+            (static_cast<uint32_t>(e4m3x2(__fmul_rn(f[2], inv), __fmul_rn(f[3], inv))) << 16);
+      q.y = static_cast<uint32_t>(e4m3x2(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv))) |
+            (static_cast<uint32_t>(e4m3x2(__fmul_rn(f[6], inv), __fmul_rn(f[7], inv))) << 16);
+    }
+    if (active) {
+      *reinterpret_cast<uint2*>(blk + v * D + sl * 8) = q;
+      if (sl == 0) reinterpret_cast<float*>(blk + p.scale_off)[v] = scale;
+    }
   }
   if (p.out == nullptr) __threadfence_system();  // peer stores performed before the kernel ends
 }
 
-// One warp per kExchangeVecPerWarp consecutive vectors of y.
+// kLanes<D> lanes per vector of y; all loads of a lane's kExchangeSteps vectors
+// first, then the dequantise-and-store pass.
 template <int D>
 __global__ void __launch_bounds__(256) exchange_unpack_kernel(ExchangeParams p) {
-  constexpr int E = D / 32, V = kExchangeVecPerWarp;
+  constexpr int LPV = kLanes<D>, VPW = 32 / LPV, S = kExchangeSteps;
   const int Tb = p.split == 0 ? p.T / p.G : p.T;
   const int Cb = p.split == 1 ? p.C / p.G : p.C;
   // y is [B][Ty][Cy][D]
   const int Ty = p.split == 1 ? p.G * Tb : Tb;
   const int Cy = p.split == 0 ? p.G * Cb : Cb;
-  const long long vec0 = (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * V;
-  const int lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31, sub = lane / LPV, sl = lane - sub * LPV;
   const long long n_vec = static_cast<long long>(p.B) * Ty * Cy;
-  uint32_t raw[V][E / 2];  // bf16 words, or the E code bytes in raw[k][0] (fp8)
-  float scale[V];
-  int cy = 0, ty = 0, b = 0;  // of the first vector once, then stepped (as in pack)
-  if (vec0 < n_vec) {
-    cy = static_cast<int>(vec0 % Cy);
-    const long long bt = vec0 / Cy;
+  const long long base =
+      (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * kExchangeVecPerWarp<D>;
+  int cy = 0, ty = 0, b = 0;  // of the lane's first vector once, then stepped
+  if (base + sub < n_vec) {
+    const long long vec = base + sub;
+    cy = static_cast<int>(vec % Cy);
+    const long long bt = vec / Cy;
     ty = static_cast<int>(bt % Ty);
     b = static_cast<int>(bt / Ty);
   }
+  uint4 raw[S];  // 8 bf16 values, or the 8 code bytes in .x/.y (fp8)
+  float scale[S];
 #pragma unroll
-  for (int k = 0; k < V; ++k) {
-    const long long vec = vec0 + k;
-    if (vec >= n_vec) break;
-    if (k > 0 && ++cy == Cy) {
-      cy = 0;
-      if (++ty == Ty) {
-        ty = 0;
-        ++b;
-      }
-    }
-    int s, tl = ty, cl = cy;
+  for (int s = 0; s < S; ++s) {
+    if (s > 0) exchange_step(VPW, Cy, Ty, b, ty, cy);
+    raw[s] = make_uint4(0u, 0u, 0u, 0u);
+    scale[s] = 0.f;
+    if (base + s * VPW + sub >= n_vec) continue;
+    int src, tl = ty, cl = cy;  // sending rank, and the position in its block
     if (p.split == 1) {
-      s = ty / Tb;
-      tl = ty - s * Tb;
+      src = ty / Tb;
+      tl = ty - src * Tb;
     } else {
-      s = cy / Cb;
-      cl = cy - s * Cb;
+      src = cy / Cb;
+      cl = cy - src * Cb;
     }
     const long long v = (static_cast<long long>(b) * Tb + tl) * Cb + cl;
-    const uint8_t* blk = p.in + s * p.block_bytes;
+    const uint8_t* blk = p.in + src * p.block_bytes;
     if (!p.fp8) {
-      const uint32_t* src = reinterpret_cast<const uint32_t*>(
-          reinterpret_cast<const __nv_bfloat16*>(blk) + v * D + lane * E);
-#pragma unroll
-      for (int i = 0; i < E / 2; ++i) raw[k][i] = src[i];
+      raw[s] = ld_nc_v4(reinterpret_cast<const __nv_bfloat16*>(blk) + v * D + sl * 8);
     } else {
-      scale[k] = reinterpret_cast<const float*>(blk + p.scale_off)[v];
-      const uint8_t* codes = blk + v * D + lane * E;
-      if constexpr (E == 4)
-        raw[k][0] = *reinterpret_cast<const uint32_t*>(codes);
-      else
-        raw[k][0] = *reinterpret_cast<const uint16_t*>(codes);
+      scale[s] = __ldg(reinterpret_cast<const float*>(blk + p.scale_off) + v);
+      const uint2 q = __ldg(reinterpret_cast<const uint2*>(blk + v * D + sl * 8));
+      raw[s].x = q.x;
+      raw[s].y = q.y;
     }
   }
 #pragma unroll
-  for (int k = 0; k < V; ++k) {
-    const long long vec = vec0 + k;
-    if (vec >= n_vec) break;
-    uint32_t* out = reinterpret_cast<uint32_t*>(p.y + vec * D + lane * E);
-    if (!p.fp8) {
+  for (int s = 0; s < S; ++s) {
+    const long long vec = base + s * VPW + sub;
+    if (vec >= n_vec) continue;
+    uint4 o = raw[s];
+    if (p.fp8) {
+      const uint32_t q2[2] = {raw[s].x, raw[s].y};
+      uint32_t r[4];
 #pragma unroll
-      for (int i = 0; i < E / 2; ++i) out[i] = raw[k][i];
-      continue;
+      for (int i = 0; i < 4; ++i) {
+        const float2 fv = e4m3x2_to_f32(static_cast<uint16_t>(q2[i / 2] >> (16 * (i & 1))));
+        r[i] = ptx::pack_bf16x2(__fmul_rn(fv.x, scale[s]), __fmul_rn(fv.y, scale[s]));
+      }
+      o = make_uint4(r[0], r[1], r[2], r[3]);
     }
-#pragma unroll
-    for (int i = 0; i < E / 2; ++i) {
-      const float2 fv = e4m3x2_to_f32(static_cast<uint16_t>(raw[k][0] >> (16 * i)));
-      out[i] = ptx::pack_bf16x2(__fmul_rn(fv.x, scale[k]), __fmul_rn(fv.y, scale[k]));
-    }
+    st_v4(p.y + vec * D + sl * 8, o);
   }
 }
 

@@ -84,19 +84,19 @@ __device__ __forceinline__ void st_v4(void* p, uint4 v) {
                : "memory");
 }
 
-// Tokens per block of rope_transpose_kernel: each thread issues the loads of all
-// of them before the first store, so enough bytes are in flight to cover HBM
-// latency (one token per thread leaves the copy latency-bound at about half the
-// bandwidth).
-constexpr int kRopeTokensPerBlock = 4;
-
-// Block x covers tokens (b, l) = kRopeTokensPerBlock * x .. + kRopeTokensPerBlock - 1
-// of the flattened [B * L] index; thread t moves 16-byte chunk t % (D/8) of head
-// t / (D/8) of each. blockIdx.y: 0 = K (bf16 in, rotated, fp16 out), 1 = V (bf16,
-// copied; rotated like K when second_is_key). Loads are fully coalesced (a
+// Rotate-and-transpose of whole frame rows. Block x covers tokens x0 .. x0 + XT - 1
+// (x0 = segment * XT, clipped to the row) of one frame row (b, f, y), so the
+// frame, the row and their RoPE table entries are per-block constants and a
+// token's column is x0 + k: the per-token index arithmetic is an add, and only
+// the column band's (cos, sin) is read per token. Thread t moves 16-byte chunk
+// t % (D/8) of head t / (D/8) of every token of the segment; it issues the loads
+// of all XT tokens before the first store, so enough bytes are in flight to
+// cover HBM latency. blockIdx.y: 0 = K (bf16 in, rotated, fp16 out), 1 = V
+// (bf16, copied; rotated like K when second_is_key). Loads are coalesced (a
 // token's H*D values are contiguous); each head's 2*D bytes are stored
 // contiguously into its [B, H, L_out, D] plane.
-__global__ void rope_transpose_kernel(AppendParams p) {
+template <int XT>
+__global__ void __launch_bounds__(XT >= 16 ? 512 : 1024) rope_transpose_kernel(AppendParams p) {
   const int vec_per_head = p.D >> 3;
   const int t = threadIdx.x;
   if (t >= p.H * vec_per_head) return;
@@ -104,29 +104,65 @@ __global__ void rope_transpose_kernel(AppendParams p) {
   const __nv_bfloat16* in = is_v ? p.v_in : p.k_in;
   __nv_bfloat16* out = is_v ? p.v_out : p.k_out;
   if (in == nullptr) return;
+  const RopeTables& rt = p.rope;
+  const int n_seg = (rt.tok_w + XT - 1) / XT;
+  const int row = blockIdx.x / n_seg;  // frame row over [B][L / tok_w]
+  const int x0 = (blockIdx.x - row * n_seg) * XT;
+  const int nx = min(XT, rt.tok_w - x0);
+  const int rows_per_b = p.L / rt.tok_w;
+  const int b = row / rows_per_b, fy = row - b * rows_per_b;
   const int h = t / vec_per_head, c = t - h * vec_per_head;
-  const int n_tok = p.B * p.L;
-  const int tok0 = blockIdx.x * kRopeTokensPerBlock;
-  bool saturated = false;
-  uint4 v[kRopeTokensPerBlock];
+  const int l0 = fy * rt.tok_w + x0;
+  const size_t hd = static_cast<size_t>(p.H) * p.D;
+  const size_t src_off = (static_cast<size_t>(b) * p.L + l0) * hd + static_cast<size_t>(h) * p.D + c * 8;
+  const size_t dst_off = ((static_cast<size_t>(b) * p.H + h) * p.L_out + l0) * p.D + c * 8;
+  const __nv_bfloat16* src = in + src_off;
+  __nv_bfloat16* dst = out + dst_off;
+  uint4 v[XT];
 #pragma unroll
-  for (int k = 0; k < kRopeTokensPerBlock; ++k) {
-    const int tok = tok0 + k;
-    if (tok < n_tok) v[k] = ld_nc_v4(in + (static_cast<size_t>(tok) * p.H + h) * p.D + c * 8);
+  for (int k = 0; k < XT; ++k)
+    if (k < nx && SA_IN_BOUNDS(p.status, src_off + k * hd + 8, p.in_elems))
+      v[k] = ld_nc_v4(src + k * hd);
+  if (is_v && !p.second_is_key) {
+#pragma unroll
+    for (int k = 0; k < XT; ++k)
+      if (k < nx && SA_IN_BOUNDS(p.status, dst_off + k * p.D + 8, p.out_elems))
+        st_v4(dst + k * p.D, v[k]);
+    return;
   }
+  // The 4 pairs of this thread's chunk: a temporal or row-band pair's (cos, sin)
+  // is fixed for the block; a column-band pair's is read per token (wcol >= 0).
+  const int f = fy / rt.tok_h, y = fy - f * rt.tok_h;
+  float2 cs[4];
+  int wcol[4];
 #pragma unroll
-  for (int k = 0; k < kRopeTokensPerBlock; ++k) {
-    const int tok = tok0 + k;
-    if (tok >= n_tok) break;
-    const int b = tok / p.L, l = tok - b * p.L;
-    if (!is_v || p.second_is_key) {
-      const int f = l / p.rope.frame_tokens;
-      const int y = (l / p.rope.tok_w) % p.rope.tok_h;
-      const int x = l % p.rope.tok_w;
-      saturated |= pair_norm_exceeds_f16(v[k]);
-      v[k] = rope_chunk(v[k], c, p.rope, f, y, x);
+  for (int j = 0; j < 4; ++j) {
+    int pr = 4 * c + j;
+    wcol[j] = -1;
+    if (pr < rt.dt2) {
+      cs[j] = __ldg(&rt.t[f * rt.dt2 + pr]);
+    } else if ((pr -= rt.dt2) < rt.dh2) {
+      cs[j] = __ldg(&rt.h[y * rt.dh2 + pr]);
+    } else {
+      wcol[j] = pr - rt.dh2;
+      cs[j] = make_float2(1.f, 0.f);
     }
-    st_v4(out + ((static_cast<size_t>(b) * p.H + h) * p.L_out + l) * p.D + c * 8, v[k]);
+  }
+  bool saturated = false;
+#pragma unroll
+  for (int k = 0; k < XT; ++k) {
+    if (k >= nx) break;
+    const int xo = (x0 + k) * rt.dw2;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (wcol[j] >= 0) cs[j] = __ldg(&rt.w[xo + wcol[j]]);
+    saturated |= pair_norm_exceeds_f16(v[k]);
+    uint4 r;
+    r.x = rope_pair(v[k].x, cs[0]);
+    r.y = rope_pair(v[k].y, cs[1]);
+    r.z = rope_pair(v[k].z, cs[2]);
+    r.w = rope_pair(v[k].w, cs[3]);
+    if (SA_IN_BOUNDS(p.status, dst_off + k * p.D + 8, p.out_elems)) st_v4(dst + k * p.D, r);
   }
   if (saturated) atomicOr(p.status, kDevWarnSaturated);
 }

@@ -406,11 +406,18 @@ int launch_rope_transpose(sa_handle* h, const void* K, const void* V, __nv_bfloa
   ap.second_is_key = second_is_key ? 1 : 0;
   ap.rope = h->rope();
   ap.status = h->status();
+  ap.in_elems = 1ULL * d.B * rows * d.H * d.D;
+  ap.out_elems = 1ULL * d.B * d.H * L_out * d.D;
+  // One block per segment of XT tokens of a frame row (rows = whole frames);
+  // 16 tokens a thread while the block fits the 512-thread register budget.
   const int threads = static_cast<int>(align_up(static_cast<size_t>(d.H) * d.D / 8, 32));
-  const long long n_tok = 1LL * d.B * rows;
-  dim3 grid(static_cast<unsigned>((n_tok + sa::kRopeTokensPerBlock - 1) / sa::kRopeTokensPerBlock),
-            V != nullptr ? 2 : 1);
-  sa::rope_transpose_kernel<<<grid, threads, 0, s>>>(ap);
+  const int xt = threads <= 512 ? 16 : 8;
+  const long long frame_rows = 1LL * d.B * (rows / d.tw);
+  dim3 grid(static_cast<unsigned>(frame_rows * ((d.tw + xt - 1) / xt)), V != nullptr ? 2 : 1);
+  if (xt == 16)
+    sa::rope_transpose_kernel<16><<<grid, threads, 0, s>>>(ap);
+  else
+    sa::rope_transpose_kernel<8><<<grid, threads, 0, s>>>(ap);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
     return h->fail(SA_ERR_CUDA, std::string("append launch: ") + cudaGetErrorString(e));
@@ -517,6 +524,13 @@ void fill_common(sa_handle* h, int tier, int n_frames, bool source, const void* 
   ap->scale_log2 = d.scale * 1.4426950408889634f;
   ap->rope = h->rope();
   ap->status = h->status();
+  ap->q_elems = 1ULL * d.B * ap->L * d.H * d.D;
+  ap->lse_elems = 1ULL * d.B * d.H * ap->L;
+  ap->bits_words = d.bits_bytes / sizeof(unsigned long long);
+  ap->split_rows = 1ULL * sa::kMaxSplitSlots * 2 * 2 * 128;
+  ap->cache_elems = 2ULL * (d.S + d.R) * d.chunk_elems;
+  ap->kcur_elems = 2ULL * d.chunk_elems;
+  ap->ref_elems = 2ULL * d.ref_elems;
 }
 
 int check_attend_ptrs(sa_handle* h, const void* Q, const void* Vc, const void* O,
@@ -623,6 +637,9 @@ int attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final
       for (int g = 0; g < ap.n_groups; ++g) bp.n_k += (ap.groups[g].len + 127) / 128;
       bp.n_words = (bp.n_k + 63) / 64;
       bp.rows = 1LL * d.B * d.H * ((ap.L + 127) / 128);
+      bp.status = h->status();
+      bp.mask_bytes = static_cast<unsigned long long>(bp.rows) * bp.n_k;
+      bp.bits_words = d.bits_bytes / sizeof(unsigned long long);
       if (static_cast<size_t>(bp.rows) * bp.n_words * sizeof(unsigned long long) > d.bits_bytes)
         return h->fail(SA_ERR_UNSUPPORTED, "block mask larger than the bit-row region");
       sa::block_bits_kernel<<<static_cast<unsigned>((bp.rows + 7) / 8), 256, 0, s>>>(bp);
@@ -782,6 +799,7 @@ int attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc, 
   AttendParams ap;
   fill_common(h, tier, d.F, false, Q, Vc, O, lse, &ap);
   ap.k_cur = keys;
+  ap.kcur_elems = SA_NOALLOC_MAX_KEY_BYTES / sizeof(__nv_bfloat16);
   ap.split_ok = 0;  // no scratch but the fixed key array: no split tail
 
   // Every element of the scratch that the attention reads is written first by
@@ -882,7 +900,8 @@ bool exchange_layout(int B, int T, int C, int D, int G, int split, int payload,
 
 int launch_exchange(bool pack, sa::ExchangeParams& ep, sa_stream stream) {
   const long long n_vec = 1LL * ep.B * ep.T * ep.C;  // vectors of x (pack) and of y (unpack)
-  const long long per_block = 8LL * sa::kExchangeVecPerWarp;  // 8 warps a block
+  const long long per_block =
+      8LL * (ep.D == 128 ? sa::kExchangeVecPerWarp<128> : sa::kExchangeVecPerWarp<64>);
   const unsigned grid = static_cast<unsigned>((n_vec + per_block - 1) / per_block);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (pack)
@@ -1429,6 +1448,9 @@ SA_API int sa_get_status(sa_handle* h, sa_stream stream) {
     return h->fail(SA_ERR_CUDA, std::string("reading the status word: ") +
                                     cudaGetErrorString(cudaGetLastError()));
   if (word & sa::kDevErrTimeout) return h->fail(SA_ERR_TIMEOUT, "a kernel gave up a bounded wait");
+  if (word & sa::kDevErrBounds)
+    return h->fail(SA_ERR_BOUNDS, "a kernel of the checked build skipped an access past the end "
+                                  "of a buffer");
   if (word & sa::kDevWarnSaturated)
     return h->fail(SA_ERR_RANGE,
                    "a Q or K pair had a norm above 65504 and was saturated to fp16 for the "
@@ -1440,6 +1462,14 @@ SA_API const char* sa_last_error(const sa_handle* h) {
   return h != nullptr ? h->err.c_str() : g_error.c_str();
 }
 
+SA_API int sa_build_info(void) {
+#ifdef SA_DEVICE_CHECKS
+  return SA_BUILD_DEVICE_CHECKS;
+#else
+  return 0;
+#endif
+}
+
 SA_API const char* sa_status_string(int status) {
   switch (status) {
     case SA_OK: return "SA_OK";
@@ -1449,6 +1479,7 @@ SA_API const char* sa_status_string(int status) {
     case SA_ERR_CUDA: return "SA_ERR_CUDA";
     case SA_ERR_TIMEOUT: return "SA_ERR_TIMEOUT";
     case SA_ERR_RANGE: return "SA_ERR_RANGE";
+    case SA_ERR_BOUNDS: return "SA_ERR_BOUNDS";
     default: return "SA_ERR_UNKNOWN";
   }
 }

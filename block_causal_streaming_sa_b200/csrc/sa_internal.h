@@ -24,6 +24,26 @@ constexpr int kModeAligned = 2;
 // its rotated values were saturated for the score MMA.
 constexpr unsigned kDevErrTimeout = 1u;
 constexpr unsigned kDevWarnSaturated = 2u;
+constexpr unsigned kDevErrBounds = 4u;
+
+// Device-side bounds checks of the checked build (libsa_checked.so, compiled
+// with SA_DEVICE_CHECKS): before a kernel reads or writes global memory
+// directly, SA_IN_BOUNDS(status, end, size) compares the end of the access (one
+// past its last element) with the buffer's size; an access past the end sets
+// kDevErrBounds in the status word and is skipped. The release build compiles
+// every check to `true`. (TMA loads need none: the tensor maps carry the
+// extents and fill out-of-range boxes with zeros.)
+#ifdef SA_DEVICE_CHECKS
+__device__ __forceinline__ bool in_bounds(unsigned* status, unsigned long long end,
+                                          unsigned long long size) {
+  if (end <= size) return true;
+  atomicOr(status, kDevErrBounds);
+  return false;
+}
+#define SA_IN_BOUNDS(status, end, size) ::sa::in_bounds((status), (end), (size))
+#else
+#define SA_IN_BOUNDS(status, end, size) true
+#endif
 
 // fp32 (cos, sin) tables of the three RoPE bands (reading: bands [t | h | w] of
 // D - 4*(D/6), 2*(D/6), 2*(D/6) dims, pair i of a band of size d turned by
@@ -50,7 +70,8 @@ struct AppendParams {
   int L_out;  // rows per output plane
   int second_is_key;
   RopeTables rope;
-  unsigned* status;  // device status word (kDevWarnSaturated)
+  unsigned* status;  // device status word (kDevWarnSaturated, kDevErrBounds)
+  unsigned long long in_elems, out_elems;  // sizes of each input and output tensor
 };
 
 // One attended key group: the reference image first (if set), then the
@@ -96,6 +117,10 @@ struct AttendParams {
   float* split_lse;  // [slot][query tile][half][128 rows]
   int* split_sem;    // [slot][query tile][128 rows], zero between launches
   int split_ok;
+  // Buffer sizes for the checked build's bounds checks (elements): Q and O, lse,
+  // bit-row words, split-tail rows; for the SIMT kernel the key sources too.
+  unsigned long long q_elems, lse_elems, bits_words, split_rows;
+  unsigned long long cache_elems, kcur_elems, ref_elems;
   int debug_stall_producer;  // test hook: 1 = the TMA producer issues nothing, so the
                              // MMA warp's bounded wait runs out (timeout path)
 };

@@ -72,8 +72,10 @@ typedef enum {
   SA_ERR_UNSUPPORTED = 3,  /* valid request the library does not serve (e.g. D) */
   SA_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed */
   SA_ERR_TIMEOUT = 5,      /* a kernel gave up a bounded wait (device status) */
-  SA_ERR_RANGE = 6         /* an operand left the fp16 range of the score MMA and
+  SA_ERR_RANGE = 6,        /* an operand left the fp16 range of the score MMA and
                               was saturated (device status; outputs degraded) */
+  SA_ERR_BOUNDS = 7        /* checked build only: a kernel skipped an access past
+                              the end of a buffer (a library bug; device status) */
 } sa_status;
 
 typedef enum { SA_TIER_NOISY = 0, SA_TIER_CLEAN = 1 } sa_tier;
@@ -408,14 +410,27 @@ SA_API int sa_slot_of(const sa_config* cfg, int32_t chunk);
 
 /* Wait for `stream`, then read and return the device status word: SA_OK;
  * SA_ERR_TIMEOUT if a kernel gave up a bounded wait since the last reset;
- * else SA_ERR_RANGE if a rotated Q or K pair of some call since the last reset
- * had a norm above 65504 and was saturated to fp16 (the outputs were computed
- * with the saturated values). */
+ * else SA_ERR_BOUNDS (checked build only, see sa_build_info) if a kernel
+ * skipped an out-of-range access; else SA_ERR_RANGE if a rotated Q or K pair
+ * of some call since the last reset had a norm above 65504 and was saturated
+ * to fp16 (the outputs were computed with the saturated values). */
 SA_API int sa_get_status(sa_handle* h, sa_stream stream);
 
 /* Text of the handle's last error (never NULL); with h == NULL, of the last
  * error of a call that had no handle yet (sa_create). */
 SA_API const char* sa_last_error(const sa_handle* h);
+
+/* Build flags of the loaded library: SA_BUILD_DEVICE_CHECKS is set in the
+ * checked build (libsa_checked.so, the same sources compiled with
+ * SA_DEVICE_CHECKS): there every kernel of the attention path (key staging,
+ * appends, the reference image, mask packing, the tensor-core and SIMT
+ * attention) compares the end of each direct global load or store with the
+ * size of its buffer before making it; an access past the end is skipped and
+ * recorded in the device status word (sa_get_status -> SA_ERR_BOUNDS). A
+ * debugging aid in place of a memory checker; the release build (libsa.so)
+ * has no checks. Host only. */
+#define SA_BUILD_DEVICE_CHECKS 1
+SA_API int sa_build_info(void);
 
 /* Name of an sa_status value. */
 SA_API const char* sa_status_string(int status);

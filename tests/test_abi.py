@@ -202,3 +202,18 @@ def test_debug_layout_and_host_pointers_without_a_gpu():
         sa.sa_exchange_pack(x.data_ptr(), 1, 8, 4, 64, 2, 1, sa.SA_PAYLOAD_FP8, buf.data_ptr())
     assert e.value.status == sa.SA_ERR_INVALID_ARG
     assert "exchange: x" in sa.last_error()
+
+
+def test_checked_build_exports_the_same_calls_and_says_so():
+    """libsa_checked.so (device-side bounds checks) exports every declared call,
+    and sa_build_info tells the two builds apart."""
+    import os
+
+    from block_causal_streaming_sa_b200 import build
+
+    assert os.path.exists(build.LIB_CHECKED), "build() makes both libraries"
+    checked = ctypes.CDLL(build.LIB_CHECKED)
+    for name in sa.header_symbols():
+        assert hasattr(checked, name), name
+    assert checked.sa_build_info() == sa.SA_BUILD_DEVICE_CHECKS
+    assert sa.lib().sa_build_info() == 0
