@@ -147,9 +147,9 @@ __device__ __noinline__ void epilogue(const AttendParams& p, uint32_t tO, bool a
   uint4* dst = reinterpret_cast<uint4*>(p.o + row_off);
   // checked build: the row of O and the lse entry lie inside their buffers
   valid = valid && SA_IN_BOUNDS(p.status, row_off + D, p.q_elems);
-  const bool lse_ok =
-      p.lse != nullptr && SA_IN_BOUNDS(p.status, static_cast<unsigned long long>(lse_idx) + 1,
-                                       p.lse_elems);
+  const bool lse_ok = valid && p.lse != nullptr &&
+                      SA_IN_BOUNDS(p.status, static_cast<unsigned long long>(lse_idx) + 1,
+                                   p.lse_elems);
   if (half < 0) {
 #pragma unroll 1
     for (int j = 0; j < D / 32; ++j) {

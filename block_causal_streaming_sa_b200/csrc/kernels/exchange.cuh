@@ -88,8 +88,8 @@ __device__ __forceinline__ float2 e4m3x2_to_f32(uint16_t v) {
 template <int D>
 constexpr int kLanes = D / 8;
 constexpr int kExchangeSteps = 4;
-template <int D>
-constexpr int kExchangeVecPerWarp = (32 / kLanes<D>) * kExchangeSteps;
+template <int D, int S = kExchangeSteps>
+constexpr int kExchangeVecPerWarp = (32 / kLanes<D>) * S;
 
 // Advance a (b, t, c) position over [B][T][C] by `step` vectors (step >= 1).
 __device__ __forceinline__ void exchange_step(int step, int C, int T, int& b, int& t, int& c) {
@@ -105,13 +105,13 @@ __device__ __forceinline__ void exchange_step(int step, int C, int T, int& b, in
 
 // kLanes<D> lanes per vector of x: the amax of a vector is reduced over its lanes
 // by shuffles; lane 0 of the vector writes its scale.
-template <int D>
+template <int D, int S = kExchangeSteps>
 __global__ void __launch_bounds__(256) exchange_pack_kernel(ExchangeParams p) {
-  constexpr int LPV = kLanes<D>, VPW = 32 / LPV, S = kExchangeSteps;
+  constexpr int LPV = kLanes<D>, VPW = 32 / LPV;
   const int lane = threadIdx.x & 31, sub = lane / LPV, sl = lane - sub * LPV;
   const long long n_vec = static_cast<long long>(p.B) * p.T * p.C;
   const long long base =
-      (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * kExchangeVecPerWarp<D>;
+      (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * kExchangeVecPerWarp<D, S>;
   uint4 w[S];
 #pragma unroll
   for (int s = 0; s < S; ++s) {
@@ -172,9 +172,9 @@ __global__ void __launch_bounds__(256) exchange_pack_kernel(ExchangeParams p) {
 
 // kLanes<D> lanes per vector of y; all loads of a lane's kExchangeSteps vectors
 // first, then the dequantise-and-store pass.
-template <int D>
+template <int D, int S = kExchangeSteps>
 __global__ void __launch_bounds__(256) exchange_unpack_kernel(ExchangeParams p) {
-  constexpr int LPV = kLanes<D>, VPW = 32 / LPV, S = kExchangeSteps;
+  constexpr int LPV = kLanes<D>, VPW = 32 / LPV;
   const int Tb = p.split == 0 ? p.T / p.G : p.T;
   const int Cb = p.split == 1 ? p.C / p.G : p.C;
   // y is [B][Ty][Cy][D]
@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(256) exchange_unpack_kernel(ExchangeParams p) 
   const int lane = threadIdx.x & 31, sub = lane / LPV, sl = lane - sub * LPV;
   const long long n_vec = static_cast<long long>(p.B) * Ty * Cy;
   const long long base =
-      (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * kExchangeVecPerWarp<D>;
+      (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * kExchangeVecPerWarp<D, S>;
   int cy = 0, ty = 0, b = 0;  // of the lane's first vector once, then stepped
   if (base + sub < n_vec) {
     const long long vec = base + sub;

@@ -408,16 +408,13 @@ int launch_rope_transpose(sa_handle* h, const void* K, const void* V, __nv_bfloa
   ap.status = h->status();
   ap.in_elems = 1ULL * d.B * rows * d.H * d.D;
   ap.out_elems = 1ULL * d.B * d.H * L_out * d.D;
-  // One block per segment of XT tokens of a frame row (rows = whole frames);
-  // 16 tokens a thread while the block fits the 512-thread register budget.
+  // One block per segment of sa::kRopeSegment tokens of a frame row (rows =
+  // whole frames).
   const int threads = static_cast<int>(align_up(static_cast<size_t>(d.H) * d.D / 8, 32));
-  const int xt = threads <= 512 ? 16 : 8;
   const long long frame_rows = 1LL * d.B * (rows / d.tw);
-  dim3 grid(static_cast<unsigned>(frame_rows * ((d.tw + xt - 1) / xt)), V != nullptr ? 2 : 1);
-  if (xt == 16)
-    sa::rope_transpose_kernel<16><<<grid, threads, 0, s>>>(ap);
-  else
-    sa::rope_transpose_kernel<8><<<grid, threads, 0, s>>>(ap);
+  const long long n_seg = (d.tw + sa::kRopeSegment - 1) / sa::kRopeSegment;
+  dim3 grid(static_cast<unsigned>(frame_rows * n_seg), V != nullptr ? 2 : 1);
+  sa::rope_transpose_kernel<sa::kRopeSegment><<<grid, threads, 0, s>>>(ap);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
     return h->fail(SA_ERR_CUDA, std::string("append launch: ") + cudaGetErrorString(e));
