@@ -466,6 +466,19 @@ class Ranks:
             self.dist.destroy_process_group()
 
 
+def append_line(append_ms, append_gbs, launch_ms, launch_bytes, hbm):
+    """The `append` object: one append launch on its own (K and V of one tier, each
+    read once and written once: launch_bytes) against the HBM peak, and the whole
+    chunk's appends (every layer, both tiers, kernel boundaries included)."""
+    out = {"chunk_ms": statistics.fmean(append_ms), "chunk_GB_per_s": append_gbs,
+           "chunk_frac_of_hbm": append_gbs / hbm, "bytes_per_launch": launch_bytes}
+    if launch_ms:
+        t = statistics.fmean(launch_ms)
+        out.update({"ms": t, "GB_per_s": launch_bytes / (t * 1e-3) / 1e9,
+                    "frac_of_hbm": launch_bytes / (t * 1e-3) / 1e9 / hbm})
+    return out
+
+
 def whole_job_tflops(flops_per_rank, ms_max, world):
     """Aggregate throughput: the work of all ranks over the slowest rank's time."""
     return flops_per_rank * world / (ms_max * 1e-3) / 1e12
@@ -539,16 +552,25 @@ def run_ours(args, w):
     attends_per_chunk = steps_per_chunk * w.layers
     appends_per_chunk = 2 * w.layers
 
-    def append_all(s):
+    def append_all(s, launch_ev=None):
+        """The chunk's appends; launch_ev = three events around the first layer's two
+        append launches (each launch timed on its own)."""
         if args.ulysses:
             for layer in layers:
                 layer.append(sa.SA_TIER_NOISY, s["Kn"], s["Vn"])
                 layer.append(sa.SA_TIER_CLEAN, s["Kcl"], s["Vcl"])
             return
-        for layer in layers:
+        for li, layer in enumerate(layers):
             h = layer.handle
+            timed = launch_ev is not None and li == 0
+            if timed:
+                launch_ev[0].record(stream)
             sa.sa_append_chunk(h, sa.SA_TIER_NOISY, s["Kn"].data_ptr(), s["Vn"].data_ptr(), sp)
+            if timed:
+                launch_ev[1].record(stream)
             sa.sa_append_chunk(h, sa.SA_TIER_CLEAN, s["Kcl"].data_ptr(), s["Vcl"].data_ptr(), sp)
+            if timed:
+                launch_ev[2].record(stream)
 
     block_mask = None
     if args.sparsity > 0:
@@ -609,7 +631,7 @@ def run_ours(args, w):
                 a += 1
         if ev is not None:
             ev[2].record(stream)
-        append_all(s)
+        append_all(s, ev[4] if ev is not None else None)
         if ev is not None:
             ev[3].record(stream)
 
@@ -623,7 +645,7 @@ def run_ours(args, w):
 
         mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
         evs = [([mk() for _ in range(attends_per_chunk)], [mk() for _ in range(attends_per_chunk)],
-                mk(), mk()) for _ in range(args.steps)]
+                mk(), mk(), [mk(), mk(), mk()]) for _ in range(args.steps)]
         start, stop = mk(), mk()
         clocks = ClockSampler(bus_id_of(dev)) if rank == 0 else None
         barrier()
@@ -643,6 +665,9 @@ def run_ours(args, w):
         ms_local = start.elapsed_time(stop)
         attend_ms = [e[0][k].elapsed_time(e[1][k]) for e in evs for k in range(attends_per_chunk)]
         append_ms = [e[2].elapsed_time(e[3]) for e in evs]
+        # each append launch alone (first layer's noisy and clean appends)
+        launch_ms = ([e[4][0].elapsed_time(e[4][1]) for e in evs] +
+                     [e[4][1].elapsed_time(e[4][2]) for e in evs]) if not args.ulysses else []
         assert attn.status(stream) == sa.SA_OK, "device status word reports a timeout"
 
         # End to end through the public API with host buffers: every step copies
@@ -746,6 +771,8 @@ def run_ours(args, w):
     append_bytes = appends_per_chunk * 2 * 2 * (w.batch * w.chunk_len * w.heads * w.head_dim * 2)
     # (per append of one tier: K and V, each read once and written once)
     append_gbs = append_bytes / (statistics.fmean(append_ms) * 1e-3) / 1e9
+    launch_bytes = 2 * 2 * (w.batch * w.chunk_len * w.heads * w.head_dim * 2)
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     line = {
         "metric": METRIC,
         "value": value,
@@ -774,8 +801,7 @@ def run_ours(args, w):
             "traffic": kernel_traffic("attend_tc.cuh", w.name),
             "flops_per_launch": flops, "avg_launch_ms": attend_avg,
         },
-        "append": {"ms": statistics.fmean(append_ms), "GB_per_s": append_gbs,
-                   "frac_of_hbm": append_gbs / float(peaks.get("hbm_gbs", 6650.0))},
+        "append": append_line(append_ms, append_gbs, launch_ms, launch_bytes, hbm),
         "ms_per_attention": attend_avg,
         "attention_tflops_kernel": achieved,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
