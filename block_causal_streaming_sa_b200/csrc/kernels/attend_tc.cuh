@@ -685,11 +685,14 @@ __global__ void __launch_bounds__(384, 1)
       // Sparse: the tiles flagged for this query tile only, cur being the next
       // one; frame-aligned units visit every group, the last one partly.
       // (The bit row and its end are re-derived where used: fewer live registers.)
+      // any_tile stays true in sparse mode too: a query tile without a flagged
+      // block runs no tile, keeps lsum = 0, and its epilogue writes O = 0 and
+      // lse = -inf (the tensor memory it reads is not used). A run-time any_tile
+      // made the sparse score loop spill.
       int g0 = glo, cur = 0;
-      bool any_tile = true;
+      const bool any_tile = true;
       if (kSparse) {
         cur = next_set(bit_row(w, i), gstart[glo], gstart[ghi]);
-        any_tile = cur < gstart[ghi];
         while (g0 + 1 < ghi && cur >= gstart[g0 + 1]) ++g0;
       }
 
@@ -697,17 +700,37 @@ __global__ void __launch_bounds__(384, 1)
       // shared memory for the re-turns at chunk switches.
       const uint32_t q_raw = sbase + T::kOffQRaw + (i * T::BM + r) * T::kQRawRow;
       {
+        // The row's 16-byte chunks are all requested before the first is used, and
+        // the RoPE (cos, sin) of 8 chunks at a time: two round trips to the tables
+        // per row instead of one per chunk (a work unit's start waits on these).
         const uint4* src = reinterpret_cast<const uint4*>(p.q + row_off);
         const int td0 = groups[g0].t_delta;
+        const bool q_ok = valid && SA_IN_BOUNDS(p.status, row_off + D, p.q_elems);
         bool saturated = false;
-#pragma unroll 2
-        for (int c = 0; c < D / 8; ++c) {
-          uint4 v = valid && SA_IN_BOUNDS(p.status, row_off + c * 8 + 8, p.q_elems)
-                        ? ld_nc_v4(src + c)
-                        : make_uint4(0u, 0u, 0u, 0u);
-          if (c < T::kTChunks) st_shared_v4(q_raw + c * 16, v);
-          saturated |= pair_norm_exceeds_f16(v);
-          st_shared_v4(q_smem + sw128_offset(r, c), rope_chunk(v, c, p.rope, td0 + f, y, x));
+        uint4 qv[D / 8];
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c)
+          qv[c] = q_ok ? ld_nc_v4(src + c) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int c8 = 0; c8 < D / 8; c8 += 8) {
+          float2 cs[8][4];
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) cs[cc][j] = rope_cs(p.rope, 4 * (c8 + cc) + j, td0 + f, y, x);
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            const int c = c8 + cc;
+            const uint4 v = qv[c];
+            if (c < T::kTChunks) st_shared_v4(q_raw + c * 16, v);
+            saturated |= pair_norm_exceeds_f16(v);
+            uint4 rv;
+            rv.x = rope_pair(v.x, cs[cc][0]);
+            rv.y = rope_pair(v.y, cs[cc][1]);
+            rv.z = rope_pair(v.z, cs[cc][2]);
+            rv.w = rope_pair(v.w, cs[cc][3]);
+            st_shared_v4(q_smem + sw128_offset(r, c), rv);
+          }
         }
         if (saturated) atomicOr(p.status, kDevWarnSaturated);
         ptx::fence_proxy_async_smem();
