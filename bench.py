@@ -155,7 +155,8 @@ class ClockSampler:
                 sm = n.nvmlDeviceGetClockInfo(self.dev, n.NVML_CLOCK_SM)
                 power = n.nvmlDeviceGetPowerUsage(self.dev) / 1000.0
                 bits = reasons_fn(self.dev)
-                self.samples.append((t, float(sm), float(self.max_mhz), power, int(bits)))
+                self.samples.append((t, float(sm), float(self.max_mhz), power, int(bits),
+                                     time.perf_counter()))
             except Exception:
                 pass
             time.sleep(self.PERIOD_S)
@@ -170,8 +171,9 @@ class ClockSampler:
         if self.nvml is not None:
             self.halt.set()
             self.thread.join(timeout=5)
+            # a sample counts when its queries overlap the region
             rows = [s for s in self.samples
-                    if (self.t0 is None or s[0] >= self.t0) and (self.t1 is None or s[0] <= self.t1)]
+                    if (self.t0 is None or s[5] >= self.t0) and (self.t1 is None or s[0] <= self.t1)]
             sm = [r[1] for r in rows]
             smax = [r[2] for r in rows]
             power = [r[3] for r in rows]
@@ -637,6 +639,9 @@ def run_ours(args, w):
 
     with torch.cuda.stream(stream):
         # Fill the window so every timed chunk attends to S + W chunks.
+        # the clock sampler runs from before the warm-up, so that it is in its
+        # steady state when a short timed region starts
+        clocks = ClockSampler(bus_id_of(dev)) if rank == 0 else None
         for c in range(w.sink + w.window - 1):
             append_all(pool[c % 2])
         for i in range(args.warmup):
@@ -647,7 +652,6 @@ def run_ours(args, w):
         evs = [([mk() for _ in range(attends_per_chunk)], [mk() for _ in range(attends_per_chunk)],
                 mk(), mk(), [mk(), mk(), mk()]) for _ in range(args.steps)]
         start, stop = mk(), mk()
-        clocks = ClockSampler(bus_id_of(dev)) if rank == 0 else None
         barrier()
         torch.cuda.synchronize(dev)
         if clocks is not None:

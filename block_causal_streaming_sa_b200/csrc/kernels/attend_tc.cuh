@@ -104,7 +104,8 @@ struct TcShape {
   __host__ __device__ static constexpr int PFULL(int i) { return 2 * NSTAGE + 4 + i; }
   __host__ __device__ static constexpr int OFINAL(int i) { return 2 * NSTAGE + 6 + i; }
   __host__ __device__ static constexpr int DRAIN() { return 2 * NSTAGE + 8; }
-  static constexpr int kNumBars = 2 * NSTAGE + 9;
+  __host__ __device__ static constexpr int QLOAD(int i) { return 2 * NSTAGE + 9 + i; }
+  static constexpr int kNumBars = 2 * NSTAGE + 11;
   static_assert(kNumBars * 8 <= 224, "barrier area");
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
@@ -241,6 +242,7 @@ __global__ void __launch_bounds__(384, 1)
                      const __grid_constant__ CUtensorMap tm_vcur,
                      const __grid_constant__ CUtensorMap tm_ref,
                      const __grid_constant__ CUtensorMap tm_vsrc,
+                     const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ AttendParams p) {
   using T = TcShape<D>;
   constexpr bool kSparse = kMode == kModeSparse;    // caller-flagged 128 x 128 blocks
@@ -295,6 +297,7 @@ __global__ void __launch_bounds__(384, 1)
       ptx::mbar_init(bar(T::SFULL(i)), 1);
       ptx::mbar_init(bar(T::PFULL(i)), 128);
       ptx::mbar_init(bar(T::OFINAL(i)), 1);
+      ptx::mbar_init(bar(T::QLOAD(i)), 1);
     }
     ptx::mbar_init(bar(T::DRAIN()), 1);
     *abort_flag = 0;
@@ -507,9 +510,31 @@ __global__ void __launch_bounds__(384, 1)
                        (accumulate || kk > 0) ? 1u : 0u);
         }
       };
+      // Query tile i of unit rr by TMA (rows past L read as zeros), issued here
+      // once unit rr - 1's O is final: every MMA that read the previous tile is
+      // then done, and the copy runs under that unit's epilogue. This thread has
+      // nothing else to do until the new tile is ready.
+      int q_issued[2] = {0, 0};  // units whose tile i was requested
+      ptx::tma_prefetch_desc(&tm_q);
       for (int rr = 0; ok; ++rr) {
         int w, half;
         if (!unit(rr, w, half)) break;
+        {
+          const int bh = w / n_pairs, pair = w - bh * n_pairs;
+          const int b = bh / p.H, h = bh - b * p.H;
+          for (int i = 0; i < 2 && ok; ++i) {
+            if (rr > 0) ok = ptx::mbar_wait(bar(T::OFINAL(i)), (rr - 1) & 1, abort_flag, p.status);
+            if (!ok) break;
+            const uint32_t qb = bar(T::QLOAD(i));
+            ptx::mbar_arrive_expect_tx(qb, T::kTile);
+#pragma unroll
+            for (int kb = 0; kb < T::KBLK; ++kb)
+              ptx::tma_load_4d(sbase + T::kOffQ + i * T::kTile + kb * T::kBox, &tm_q, qb, kb * 64,
+                               h, (2 * pair + i) * T::BM, b);
+            q_issued[i] = rr + 1;
+          }
+          if (!ok) break;
+        }
         const int lo = gstart[g_lo(half)], hi = gstart[g_hi(half)];
         int mo, mo1;
         mask_rows(w, mo, mo1);
@@ -517,6 +542,8 @@ __global__ void __launch_bounds__(384, 1)
         if (kAligned && u >= hi) {  // no key tile: nothing to multiply
           for (int i = 0; i < 2 && ok; ++i)
             ok = ptx::mbar_wait(bar(T::QREADY(i)), rr & 1, abort_flag, p.status);
+          if (ok)
+            for (int i = 0; i < 2; ++i) ptx::umma_commit(bar(T::OFINAL(i)));
           continue;
         }
         if constexpr (!kSparse) {
@@ -647,10 +674,14 @@ __global__ void __launch_bounds__(384, 1)
             for (int i = 0; i < 2; ++i) ptx::umma_commit(bar(T::OFINAL(i)));
         }
       }
-      // Every MMA issued so far must finish before TMEM is released.
+      // Every MMA issued so far must finish before TMEM is released, and the last
+      // query copies must land before the CTA can exit (also after an abort).
       volatile int no_abort = 0;
       ptx::umma_commit(bar(T::DRAIN()));
       ptx::mbar_wait(bar(T::DRAIN()), 0, &no_abort, p.status);
+      for (int i = 0; i < 2; ++i)
+        if (q_issued[i] > 0)
+          ptx::mbar_wait(bar(T::QLOAD(i)), (q_issued[i] - 1) & 1, &no_abort, p.status);
     }
   }
   } else {
@@ -665,7 +696,6 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t q_smem = sbase + T::kOffQ + i * T::kTile;
     uint32_t s_phase = 0;
     bool ok = true;
-    int o_units = 0;  // units whose O this warpgroup waited for (OFINAL phases)
     for (int rr = 0; ok; ++rr) {
       int w, half;
       if (!unit(rr, w, half)) break;
@@ -699,18 +729,15 @@ __global__ void __launch_bounds__(384, 1)
       // Rotated query tile for that chunk; the raw temporal chunks are kept in
       // shared memory for the re-turns at chunk switches.
       const uint32_t q_raw = sbase + T::kOffQRaw + (i * T::BM + r) * T::kQRawRow;
+      if (!ptx::mbar_wait(bar(T::QLOAD(i)), rr & 1, abort_flag, p.status)) break;
       {
-        // The row's 16-byte chunks are all requested before the first is used, and
-        // the RoPE (cos, sin) of 8 chunks at a time: two round trips to the tables
-        // per row instead of one per chunk (a work unit's start waits on these).
-        const uint4* src = reinterpret_cast<const uint4*>(p.q + row_off);
+        // Each thread turns its own row in place; the RoPE (cos, sin) of 8 chunks
+        // are fetched at a time: two round trips to the tables per row.
         const int td0 = groups[g0].t_delta;
-        const bool q_ok = valid && SA_IN_BOUNDS(p.status, row_off + D, p.q_elems);
         bool saturated = false;
         uint4 qv[D / 8];
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c)
-          qv[c] = q_ok ? ld_nc_v4(src + c) : make_uint4(0u, 0u, 0u, 0u);
+        for (int c = 0; c < D / 8; ++c) qv[c] = ld_shared_v4(q_smem + sw128_offset(r, c));
 #pragma unroll
         for (int c8 = 0; c8 < D / 8; c8 += 8) {
           float2 cs[8][4];
@@ -872,11 +899,8 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (!ok) break;
 
-      if (any_tile || kSparse) {  // sparse: committed for a tile without blocks too
-        if (!ptx::mbar_wait(bar(T::OFINAL(i)), o_units & 1, abort_flag, p.status)) break;
-        ++o_units;
-        ptx::tc_fence_after();
-      }
+      if (!ptx::mbar_wait(bar(T::OFINAL(i)), rr & 1, abort_flag, p.status)) break;
+      ptx::tc_fence_after();
       epilogue<D>(p, tO, any_tile, m, lsum, half,
                   w - (sched[0] - 1) * static_cast<int>(gridDim.x), i, r, row_off,
                   (static_cast<long long>(b) * p.H + h) * p.L + q_row, valid);

@@ -28,7 +28,7 @@ __global__ void __launch_bounds__(256) block_bits_kernel(const BlockBitsParams p
   if (row >= p.rows) return;
   const uint8_t* m = p.mask + row * p.n_k;
   unsigned long long* out = p.bits + row * p.n_words;
-  const unsigned long long m0 = static_cast<unsigned long long>(row) * p.n_k;
+  [[maybe_unused]] const unsigned long long m0 = static_cast<unsigned long long>(row) * p.n_k;
   for (int wd = 0; wd < p.n_words; ++wd) {
     const int k = wd * 64 + lane;
     const unsigned lo = __ballot_sync(

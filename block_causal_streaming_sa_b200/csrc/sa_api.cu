@@ -260,20 +260,21 @@ unsigned attend_grid(const Derived& d, int rows, int sm_count, bool split_ok) {
 
 // The attention kernel instantiations: head dim 128 / 64, dense / block-sparse.
 // Tensor maps of one launch: cache tier, key scratch, current V, reference,
-// source V (frame-aligned editing).
+// source V (frame-aligned editing), queries.
 struct AttendMaps {
   const CUtensorMap* cache;
   const CUtensorMap* kcur;
   const CUtensorMap* vcur;
   const CUtensorMap* ref;
   const CUtensorMap* vsrc;
+  const CUtensorMap* q;
 };
 
 template <int D, int kMode>
 void launch_attend_tc_t(unsigned grid, cudaStream_t s, const AttendMaps& m,
                         const AttendParams& ap) {
   sa::attend_tc_kernel<D, kMode><<<grid, sa::TcShape<D>::kThreads, sa::TcShape<D>::kSmemBytes,
-                                   s>>>(*m.cache, *m.kcur, *m.vcur, *m.ref, *m.vsrc, ap);
+                                   s>>>(*m.cache, *m.kcur, *m.vcur, *m.ref, *m.vsrc, *m.q, ap);
 }
 
 template <int D>
@@ -620,11 +621,12 @@ int attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final
     else
       sa::attend_simt_kernel<64><<<grid, 256, 0, s>>>(ap);
   } else {
-    CUtensorMap tm_v, tm_vs;
-    if (!encode_blhd(&tm_v, Vc, d, ap.L) || (aligned && !encode_blhd(&tm_vs, Vs, d, ap.L)))
-      return h->fail(SA_ERR_CUDA, "TMA descriptor for Vc / Vs failed");
+    CUtensorMap tm_v, tm_vs, tm_q;
+    if (!encode_blhd(&tm_v, Vc, d, ap.L) || (aligned && !encode_blhd(&tm_vs, Vs, d, ap.L)) ||
+        !encode_blhd(&tm_q, Q, d, ap.L))
+      return h->fail(SA_ERR_CUDA, "TMA descriptor for Q / Vc / Vs failed");
     AttendMaps maps{h->has_cache ? &h->tm_tier[tier] : &h->tm_kcur, &h->tm_kcur, &tm_v,
-                    d.RF > 0 ? &h->tm_ref : &h->tm_kcur, aligned ? &tm_vs : &tm_v};
+                    d.RF > 0 ? &h->tm_ref : &h->tm_kcur, aligned ? &tm_vs : &tm_v, &tm_q};
     if (block_mask != nullptr) {
       // Pack the mask's rows for this launch's key groups into bit rows.
       sa::BlockBitsParams bp;
@@ -789,8 +791,9 @@ int attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc, 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int tier = step_is_final ? SA_TIER_CLEAN : SA_TIER_NOISY;
 
-  CUtensorMap tm_keys, tm_v;
-  if (!encode_planes(&tm_keys, keys, d, d.L, 1LL * d.B * d.H) || !encode_blhd(&tm_v, Vc, d, d.L))
+  CUtensorMap tm_keys, tm_v, tm_q;
+  if (!encode_planes(&tm_keys, keys, d, d.L, 1LL * d.B * d.H) ||
+      !encode_blhd(&tm_v, Vc, d, d.L) || !encode_blhd(&tm_q, Q, d, d.L))
     return h->fail(SA_ERR_CUDA, "TMA descriptors for sa_attend_noalloc failed");
 
   AttendParams ap;
@@ -804,7 +807,7 @@ int attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc, 
   rc = launch_rope_transpose(h, Kc, nullptr, keys, nullptr, d.L, d.L, s);
   if (rc != SA_OK) return rc;
   AttendMaps maps{h->has_cache ? &h->tm_tier[tier] : &tm_keys, &tm_keys, &tm_v,
-                  d.RF > 0 ? &h->tm_ref : &tm_keys, &tm_v};
+                  d.RF > 0 ? &h->tm_ref : &tm_keys, &tm_v, &tm_q};
   launch_attend_tc(d.D, sa::kModeDense, attend_grid(d, d.L, h->sm_count, false), s, maps, ap);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
