@@ -49,22 +49,6 @@ struct ExchangeParams {
 
 constexpr float kE4m3Max = 448.0f;
 
-// Block g and the vector index inside it of sender vector (b, t, c).
-__device__ __forceinline__ void exchange_place(const ExchangeParams& p, int b, int t, int c,
-                                               int& g, long long& v) {
-  const int Tb = p.split == 0 ? p.T / p.G : p.T;
-  const int Cb = p.split == 1 ? p.C / p.G : p.C;
-  int tl = t, cl = c;
-  if (p.split == 0) {
-    g = t / Tb;
-    tl = t - g * Tb;
-  } else {
-    g = c / Cb;
-    cl = c - g * Cb;
-  }
-  v = (static_cast<long long>(b) * Tb + tl) * Cb + cl;
-}
-
 __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
@@ -81,160 +65,220 @@ __device__ __forceinline__ float2 e4m3x2_to_f32(uint16_t v) {
   return f;
 }
 
-// Lanes per (b, t, c) vector: each lane moves 8 elements (16 bytes of bf16), so
-// a warp holds 32 / kLanes<D> vectors at a time; every lane issues the loads of
-// kExchangeSteps such groups before its first store, so enough bytes are in
-// flight to cover memory latency.
+// Position of a vector in the exchange: batch b, rank block g, and (tl, cl), its
+// token and head inside the block (a block is [B][Tb][Cb] vectors). The pass
+// walks its own tensor in order, head fastest, and the block index is either
+// inside the token (g_inner: a head split of x, or a token split of y, where a
+// token row holds all G blocks) or outside it (a token split of x, a head split
+// of y). step(k) advances by k vectors with no division.
+struct ExchangePos {
+  int b, g, tl, cl;
+  __device__ __forceinline__ void init(unsigned vec, bool g_inner, int G, int Tb, int Cb) {
+    cl = static_cast<int>(vec % Cb);
+    unsigned r = vec / Cb;
+    if (g_inner) {
+      g = static_cast<int>(r % G);
+      r /= G;
+      tl = static_cast<int>(r % Tb);
+      b = static_cast<int>(r / Tb);
+    } else {
+      tl = static_cast<int>(r % Tb);
+      r /= Tb;
+      g = static_cast<int>(r % G);
+      b = static_cast<int>(r / G);
+    }
+  }
+  __device__ __forceinline__ void step(int k, bool g_inner, int G, int Tb, int Cb) {
+    cl += k;
+    while (cl >= Cb) {
+      cl -= Cb;
+      if (g_inner) {
+        if (++g == G) {
+          g = 0;
+          if (++tl == Tb) {
+            tl = 0;
+            ++b;
+          }
+        }
+      } else if (++tl == Tb) {
+        tl = 0;
+        if (++g == G) {
+          g = 0;
+          ++b;
+        }
+      }
+    }
+  }
+  // vector index inside its block
+  __device__ __forceinline__ long long in_block(int Tb, int Cb) const {
+    return (static_cast<long long>(b) * Tb + tl) * Cb + cl;
+  }
+};
+
+// Sixteen elements per lane: kLanes<D> = D / 16 lanes per vector, lane sl holding
+// the vector's 16-byte chunks sl and sl + kLanes<D> (so each load and store
+// instruction covers whole halves of the vectors), and kSteps<D> steps of VPW
+// vectors per warp, kVecPerWarp in all; all loads of a lane before its first
+// store, so enough bytes are in flight to cover memory latency.
 template <int D>
-constexpr int kLanes = D / 8;
-constexpr int kExchangeSteps = 4;
-template <int D, int S = kExchangeSteps>
-constexpr int kExchangeVecPerWarp = (32 / kLanes<D>) * S;
+constexpr int kLanes = D / 16;
+template <int D>
+constexpr int kSteps = 16 / (32 / kLanes<D>);
+constexpr int kVecPerWarp = 16;
 
-// Advance a (b, t, c) position over [B][T][C] by `step` vectors (step >= 1).
-__device__ __forceinline__ void exchange_step(int step, int C, int T, int& b, int& t, int& c) {
-  c += step;
-  while (c >= C) {
-    c -= C;
-    if (++t == T) {
-      t = 0;
-      ++b;
-    }
-  }
-}
-
-// kLanes<D> lanes per vector of x: the amax of a vector is reduced over its lanes
-// by shuffles; lane 0 of the vector writes its scale.
-template <int D, int S = kExchangeSteps>
+// pack: the amax of a vector is reduced over its lanes by shuffles; lane 0 of the
+// vector writes its scale. The warp's 16 vectors need 32 divisions (scale and
+// its reciprocal): lane l computes the one of vector l % 16, the scale for
+// l < 16 and the reciprocal above, so the warp runs one division in all, and
+// the results are shuffled back.
+template <int D>
 __global__ void __launch_bounds__(256) exchange_pack_kernel(ExchangeParams p) {
-  constexpr int LPV = kLanes<D>, VPW = 32 / LPV;
+  constexpr int LPV = kLanes<D>, VPW = 32 / LPV, S = kSteps<D>, NV = kVecPerWarp;
+  static_assert(VPW * S == NV && 2 * NV <= 32, "one division per lane");
   const int lane = threadIdx.x & 31, sub = lane / LPV, sl = lane - sub * LPV;
-  const long long n_vec = static_cast<long long>(p.B) * p.T * p.C;
-  const long long base =
-      (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * kExchangeVecPerWarp<D, S>;
-  uint4 w[S];
+  const unsigned n_vec = static_cast<unsigned>(p.B) * p.T * p.C;
+  const unsigned base = (blockIdx.x * 8u + (threadIdx.x >> 5)) * NV;
+  uint4 w[S][2];
 #pragma unroll
   for (int s = 0; s < S; ++s) {
-    const long long vec = base + s * VPW + sub;
-    w[s] = vec < n_vec ? ld_nc_v4(p.x + vec * D + sl * 8) : make_uint4(0u, 0u, 0u, 0u);
+    const unsigned vec = base + s * VPW + sub;
+    const __nv_bfloat16* src = p.x + static_cast<size_t>(vec) * D + sl * 8;
+    w[s][0] = vec < n_vec ? ld_nc_v4(src) : make_uint4(0u, 0u, 0u, 0u);
+    w[s][1] = vec < n_vec ? ld_nc_v4(src + LPV * 8) : make_uint4(0u, 0u, 0u, 0u);
   }
-  // (b, t, c) of this lane's first vector once (64-bit division is a long
-  // routine), then stepped
-  int c = 0, t = 0, b = 0;
-  if (base + sub < n_vec) {
-    const long long vec = base + sub;
-    c = static_cast<int>(vec % p.C);
-    const long long bt = vec / p.C;
-    t = static_cast<int>(bt % p.T);
-    b = static_cast<int>(bt / p.T);
-  }
+  const int Tb = p.split == 0 ? p.T / p.G : p.T;
+  const int Cb = p.split == 1 ? p.C / p.G : p.C;
+  const bool g_inner = p.split == 1;
+  ExchangePos pos;
+  pos.init(base + sub, g_inner, p.G, Tb, Cb);
+  float amax[S];
 #pragma unroll
   for (int s = 0; s < S; ++s) {
-    if (s > 0) exchange_step(VPW, p.C, p.T, b, t, c);
-    const bool active = base + s * VPW + sub < n_vec;
-    int g = 0;
-    long long v = 0;
-    if (active) exchange_place(p, b, t, c, g, v);
-    uint8_t* blk = p.out != nullptr ? p.out + g * p.block_bytes : p.dst[g];
-    if (!p.fp8) {
-      if (active) st_v4(reinterpret_cast<__nv_bfloat16*>(blk) + v * D + sl * 8, w[s]);
-      continue;
-    }
-    const uint32_t ww[4] = {w[s].x, w[s].y, w[s].z, w[s].w};
-    float f[8];
+    float a = 0.f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      f[2 * i] = __uint_as_float(ww[i] << 16);
-      f[2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u);
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t ww[4] = {w[s][h].x, w[s][h].y, w[s][h].z, w[s][h].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        a = fmaxf(a, fmaxf(fabsf(__uint_as_float(ww[i] << 16)),
+                           fabsf(__uint_as_float(ww[i] & 0xFFFF0000u))));
     }
-    float amax = fmaxf(fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3]))),
-                       fmaxf(fmaxf(fabsf(f[4]), fabsf(f[5])), fmaxf(fabsf(f[6]), fabsf(f[7]))));
     // every lane takes part (inactive ones with zeros): the shuffles need the full warp
 #pragma unroll
     for (int off = LPV / 2; off > 0; off >>= 1)
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    const float scale = __fdiv_rn(amax, kE4m3Max);
-    const float inv = amax > 0.f ? __fdiv_rn(kE4m3Max, amax) : 0.f;
-    uint2 q = make_uint2(0u, 0u);
-    if (scale > 0.f) {
-      q.x = static_cast<uint32_t>(e4m3x2(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv))) |
-            (static_cast<uint32_t>(e4m3x2(__fmul_rn(f[2], inv), __fmul_rn(f[3], inv))) << 16);
-      q.y = static_cast<uint32_t>(e4m3x2(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv))) |
-            (static_cast<uint32_t>(e4m3x2(__fmul_rn(f[6], inv), __fmul_rn(f[7], inv))) << 16);
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+    amax[s] = a;
+  }
+  float quot = 0.f;  // this lane's division (fp8 only)
+  if (p.fp8) {
+    const int qv = lane % NV;  // vector s * VPW + sub of the warp
+    float a = 0.f;
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+      const float as = __shfl_sync(0xffffffffu, amax[s], (qv % VPW) * LPV);
+      if (qv / VPW == s) a = as;
     }
-    if (active) {
-      *reinterpret_cast<uint2*>(blk + v * D + sl * 8) = q;
-      if (sl == 0) reinterpret_cast<float*>(blk + p.scale_off)[v] = scale;
+    const bool recip = lane >= NV;
+    quot = __fdiv_rn(recip ? kE4m3Max : a, recip ? a : kE4m3Max);
+  }
+#pragma unroll
+  for (int s = 0; s < S; ++s) {
+    if (s > 0) pos.step(VPW, g_inner, p.G, Tb, Cb);
+    const bool active = base + s * VPW + sub < n_vec;
+    const long long v = pos.in_block(Tb, Cb);
+    const int g = active ? pos.g : 0;
+    uint8_t* blk = p.out != nullptr ? p.out + g * p.block_bytes : p.dst[g];
+    if (!p.fp8) {
+      if (active) {
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(blk) + v * D + sl * 8;
+        st_v4(dst, w[s][0]);
+        st_v4(dst + LPV * 8, w[s][1]);
+      }
+      continue;
     }
+    const float scale = __shfl_sync(0xffffffffu, quot, s * VPW + sub);
+    const float inv_q = __shfl_sync(0xffffffffu, quot, NV + s * VPW + sub);
+    const float inv = amax[s] > 0.f ? inv_q : 0.f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t ww[4] = {w[s][h].x, w[s][h].y, w[s][h].z, w[s][h].w};
+      float f[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(ww[i] << 16);
+        f[2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u);
+      }
+      uint2 q = make_uint2(0u, 0u);
+      if (scale > 0.f) {
+        q.x = static_cast<uint32_t>(e4m3x2(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv))) |
+              (static_cast<uint32_t>(e4m3x2(__fmul_rn(f[2], inv), __fmul_rn(f[3], inv))) << 16);
+        q.y = static_cast<uint32_t>(e4m3x2(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv))) |
+              (static_cast<uint32_t>(e4m3x2(__fmul_rn(f[6], inv), __fmul_rn(f[7], inv))) << 16);
+      }
+      if (active) *reinterpret_cast<uint2*>(blk + v * D + (sl + h * LPV) * 8) = q;
+    }
+    if (active && sl == 0) reinterpret_cast<float*>(blk + p.scale_off)[v] = scale;
   }
   if (p.out == nullptr) __threadfence_system();  // peer stores performed before the kernel ends
 }
 
-// kLanes<D> lanes per vector of y; all loads of a lane's kExchangeSteps vectors
-// first, then the dequantise-and-store pass.
-template <int D, int S = kExchangeSteps>
+// unpack: kLanes<D> lanes per vector of y; all loads of a lane's vectors first,
+// then the dequantise-and-store pass.
+template <int D>
 __global__ void __launch_bounds__(256) exchange_unpack_kernel(ExchangeParams p) {
-  constexpr int LPV = kLanes<D>, VPW = 32 / LPV;
+  constexpr int LPV = kLanes<D>, VPW = 32 / LPV, S = kSteps<D>, NV = kVecPerWarp;
   const int Tb = p.split == 0 ? p.T / p.G : p.T;
   const int Cb = p.split == 1 ? p.C / p.G : p.C;
-  // y is [B][Ty][Cy][D]
-  const int Ty = p.split == 1 ? p.G * Tb : Tb;
-  const int Cy = p.split == 0 ? p.G * Cb : Cb;
+  // y is [B][Ty][Cy][D]: split 1 [B][G * Tb][Cb], split 0 [B][Tb][G * Cb]
+  const bool g_inner = p.split == 0;
   const int lane = threadIdx.x & 31, sub = lane / LPV, sl = lane - sub * LPV;
-  const long long n_vec = static_cast<long long>(p.B) * Ty * Cy;
-  const long long base =
-      (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * kExchangeVecPerWarp<D, S>;
-  int cy = 0, ty = 0, b = 0;  // of the lane's first vector once, then stepped
-  if (base + sub < n_vec) {
-    const long long vec = base + sub;
-    cy = static_cast<int>(vec % Cy);
-    const long long bt = vec / Cy;
-    ty = static_cast<int>(bt % Ty);
-    b = static_cast<int>(bt / Ty);
-  }
-  uint4 raw[S];  // 8 bf16 values, or the 8 code bytes in .x/.y (fp8)
+  const unsigned n_vec = static_cast<unsigned>(p.B) * p.T * p.C;
+  const unsigned base = (blockIdx.x * 8u + (threadIdx.x >> 5)) * NV;
+  ExchangePos pos;
+  pos.init(base + sub, g_inner, p.G, Tb, Cb);
+  uint4 raw[S][2];  // bf16 payload: the two chunks; fp8: their codes in .x/.y
   float scale[S];
 #pragma unroll
   for (int s = 0; s < S; ++s) {
-    if (s > 0) exchange_step(VPW, Cy, Ty, b, ty, cy);
-    raw[s] = make_uint4(0u, 0u, 0u, 0u);
+    if (s > 0) pos.step(VPW, g_inner, p.G, Tb, Cb);
+    raw[s][0] = raw[s][1] = make_uint4(0u, 0u, 0u, 0u);
     scale[s] = 0.f;
     if (base + s * VPW + sub >= n_vec) continue;
-    int src, tl = ty, cl = cy;  // sending rank, and the position in its block
-    if (p.split == 1) {
-      src = ty / Tb;
-      tl = ty - src * Tb;
-    } else {
-      src = cy / Cb;
-      cl = cy - src * Cb;
-    }
-    const long long v = (static_cast<long long>(b) * Tb + tl) * Cb + cl;
-    const uint8_t* blk = p.in + src * p.block_bytes;
+    const long long v = pos.in_block(Tb, Cb);
+    const uint8_t* blk = p.in + pos.g * p.block_bytes;  // block of sending rank g
     if (!p.fp8) {
-      raw[s] = ld_nc_v4(reinterpret_cast<const __nv_bfloat16*>(blk) + v * D + sl * 8);
+      const __nv_bfloat16* in = reinterpret_cast<const __nv_bfloat16*>(blk) + v * D + sl * 8;
+      raw[s][0] = ld_nc_v4(in);
+      raw[s][1] = ld_nc_v4(in + LPV * 8);
     } else {
       scale[s] = __ldg(reinterpret_cast<const float*>(blk + p.scale_off) + v);
-      const uint2 q = __ldg(reinterpret_cast<const uint2*>(blk + v * D + sl * 8));
-      raw[s].x = q.x;
-      raw[s].y = q.y;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint2 q = __ldg(reinterpret_cast<const uint2*>(blk + v * D + (sl + h * LPV) * 8));
+        raw[s][h].x = q.x;
+        raw[s][h].y = q.y;
+      }
     }
   }
 #pragma unroll
   for (int s = 0; s < S; ++s) {
-    const long long vec = base + s * VPW + sub;
+    const unsigned vec = base + s * VPW + sub;
     if (vec >= n_vec) continue;
-    uint4 o = raw[s];
-    if (p.fp8) {
-      const uint32_t q2[2] = {raw[s].x, raw[s].y};
-      uint32_t r[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 fv = e4m3x2_to_f32(static_cast<uint16_t>(q2[i / 2] >> (16 * (i & 1))));
-        r[i] = ptx::pack_bf16x2(__fmul_rn(fv.x, scale[s]), __fmul_rn(fv.y, scale[s]));
+    for (int h = 0; h < 2; ++h) {
+      uint4 o = raw[s][h];
+      if (p.fp8) {
+        const uint32_t q2[2] = {raw[s][h].x, raw[s][h].y};
+        uint32_t r[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 fv = e4m3x2_to_f32(static_cast<uint16_t>(q2[i / 2] >> (16 * (i & 1))));
+          r[i] = ptx::pack_bf16x2(__fmul_rn(fv.x, scale[s]), __fmul_rn(fv.y, scale[s]));
+        }
+        o = make_uint4(r[0], r[1], r[2], r[3]);
       }
-      o = make_uint4(r[0], r[1], r[2], r[3]);
+      st_v4(p.y + static_cast<size_t>(vec) * D + (sl + h * LPV) * 8, o);
     }
-    st_v4(p.y + vec * D + sl * 8, o);
   }
 }
 

@@ -409,13 +409,16 @@ int launch_rope_transpose(sa_handle* h, const void* K, const void* V, __nv_bfloa
   ap.status = h->status();
   ap.in_elems = 1ULL * d.B * rows * d.H * d.D;
   ap.out_elems = 1ULL * d.B * d.H * L_out * d.D;
-  // One block per segment of sa::kRopeSegment tokens of a frame row (rows =
-  // whole frames).
-  const int threads = static_cast<int>(align_up(static_cast<size_t>(d.H) * d.D / 8, 32));
+  // One block per segment of XT tokens of a frame row (rows = whole frames), a
+  // thread per (token, 16-byte chunk).
+  const int xt = d.D == 128 ? sa::kRopeTokens<128> : sa::kRopeTokens<64>;
   const long long frame_rows = 1LL * d.B * (rows / d.tw);
-  const long long n_seg = (d.tw + sa::kRopeSegment - 1) / sa::kRopeSegment;
+  const long long n_seg = (d.tw + xt - 1) / xt;
   dim3 grid(static_cast<unsigned>(frame_rows * n_seg), V != nullptr ? 2 : 1);
-  sa::rope_transpose_kernel<sa::kRopeSegment><<<grid, threads, 0, s>>>(ap);
+  if (d.D == 128)
+    sa::rope_transpose_kernel<sa::kRopeTokens<128>, sa::kRopeHeadGroup><<<grid, 256, 0, s>>>(ap);
+  else
+    sa::rope_transpose_kernel<sa::kRopeTokens<64>, sa::kRopeHeadGroup><<<grid, 256, 0, s>>>(ap);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
     return h->fail(SA_ERR_CUDA, std::string("append launch: ") + cudaGetErrorString(e));
@@ -875,8 +878,8 @@ bool exchange_layout(int B, int T, int C, int D, int G, int split, int payload,
     return false;
   }
   const long long n_vec = 1LL * B * T * C;
-  if (n_vec > (1LL << 32)) {
-    g_error = "exchange: tensor too large";
+  if (n_vec >= (1LL << 31)) {  // the kernels index vectors in 32 bits
+    g_error = "exchange: tensor too large (B*T*C must stay below 2^31 vectors)";
     return false;
   }
   const long long per_block = n_vec / G;
@@ -900,8 +903,7 @@ bool exchange_layout(int B, int T, int C, int D, int G, int split, int payload,
 
 int launch_exchange(bool pack, sa::ExchangeParams& ep, sa_stream stream) {
   const long long n_vec = 1LL * ep.B * ep.T * ep.C;  // vectors of x (pack) and of y (unpack)
-  const long long per_block =
-      8LL * (ep.D == 128 ? sa::kExchangeVecPerWarp<128> : sa::kExchangeVecPerWarp<64>);
+  const long long per_block = 8LL * sa::kVecPerWarp;  // 8 warps a block
   const unsigned grid = static_cast<unsigned>((n_vec + per_block - 1) / per_block);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (pack)
