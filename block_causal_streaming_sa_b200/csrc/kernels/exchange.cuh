@@ -117,23 +117,25 @@ struct ExchangePos {
 
 // Sixteen elements per lane: kLanes<D> = D / 16 lanes per vector, lane sl holding
 // the vector's 16-byte chunks sl and sl + kLanes<D> (so each load and store
-// instruction covers whole halves of the vectors), and kSteps<D> steps of VPW
-// vectors per warp, kVecPerWarp in all; all loads of a lane before its first
-// store, so enough bytes are in flight to cover memory latency.
+// instruction covers whole halves of the vectors), and a fixed number of vectors
+// per warp in steps of VPW = 32 / kLanes<D>; all loads of a lane before its
+// first store, so enough bytes are in flight to cover memory latency. Measured
+// on B200 (720p, 12 heads): pack with 8 vectors per warp at 4 blocks of 256
+// threads per SM (64 registers) beat 16 vectors per warp at 2 blocks (127
+// registers) by 15 %; unpack (55 registers) runs 16.
 template <int D>
 constexpr int kLanes = D / 16;
-template <int D>
-constexpr int kSteps = 16 / (32 / kLanes<D>);
-constexpr int kVecPerWarp = 16;
+constexpr int kPackVecPerWarp = 8;
+constexpr int kUnpackVecPerWarp = 16;
 
 // pack: the amax of a vector is reduced over its lanes by shuffles; lane 0 of the
-// vector writes its scale. The warp's 16 vectors need 32 divisions (scale and
-// its reciprocal): lane l computes the one of vector l % 16, the scale for
-// l < 16 and the reciprocal above, so the warp runs one division in all, and
-// the results are shuffled back.
+// vector writes its scale. The warp's NV vectors need 2 NV divisions (scale and
+// its reciprocal): lane l computes the one of vector l % NV, the scale for
+// (l / NV) even and the reciprocal for odd, so the warp runs one division in
+// all, and the results are shuffled back.
 template <int D>
-__global__ void __launch_bounds__(256) exchange_pack_kernel(ExchangeParams p) {
-  constexpr int LPV = kLanes<D>, VPW = 32 / LPV, S = kSteps<D>, NV = kVecPerWarp;
+__global__ void __launch_bounds__(256, 4) exchange_pack_kernel(ExchangeParams p) {
+  constexpr int LPV = kLanes<D>, VPW = 32 / LPV, NV = kPackVecPerWarp, S = NV / VPW;
   static_assert(VPW * S == NV && 2 * NV <= 32, "one division per lane");
   const int lane = threadIdx.x & 31, sub = lane / LPV, sl = lane - sub * LPV;
   const unsigned n_vec = static_cast<unsigned>(p.B) * p.T * p.C;
@@ -178,7 +180,7 @@ __global__ void __launch_bounds__(256) exchange_pack_kernel(ExchangeParams p) {
       const float as = __shfl_sync(0xffffffffu, amax[s], (qv % VPW) * LPV);
       if (qv / VPW == s) a = as;
     }
-    const bool recip = lane >= NV;
+    const bool recip = (lane / NV) & 1;
     quot = __fdiv_rn(recip ? kE4m3Max : a, recip ? a : kE4m3Max);
   }
 #pragma unroll
@@ -226,7 +228,7 @@ __global__ void __launch_bounds__(256) exchange_pack_kernel(ExchangeParams p) {
 // then the dequantise-and-store pass.
 template <int D>
 __global__ void __launch_bounds__(256) exchange_unpack_kernel(ExchangeParams p) {
-  constexpr int LPV = kLanes<D>, VPW = 32 / LPV, S = kSteps<D>, NV = kVecPerWarp;
+  constexpr int LPV = kLanes<D>, VPW = 32 / LPV, NV = kUnpackVecPerWarp, S = NV / VPW;
   const int Tb = p.split == 0 ? p.T / p.G : p.T;
   const int Cb = p.split == 1 ? p.C / p.G : p.C;
   // y is [B][Ty][Cy][D]: split 1 [B][G * Tb][Cb], split 0 [B][Tb][G * Cb]

@@ -903,7 +903,7 @@ bool exchange_layout(int B, int T, int C, int D, int G, int split, int payload,
 
 int launch_exchange(bool pack, sa::ExchangeParams& ep, sa_stream stream) {
   const long long n_vec = 1LL * ep.B * ep.T * ep.C;  // vectors of x (pack) and of y (unpack)
-  const long long per_block = 8LL * sa::kVecPerWarp;  // 8 warps a block
+  const long long per_block = 8LL * (pack ? sa::kPackVecPerWarp : sa::kUnpackVecPerWarp);  // 8 warps
   const unsigned grid = static_cast<unsigned>((n_vec + per_block - 1) / per_block);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (pack)
