@@ -665,6 +665,12 @@ def run_ours(args, w):
             clocks.mark_stop()
         torch.cuda.synchronize(dev)
         clock_info = clocks.stop() if clocks is not None else None
+        # the SM clock the last timed attention kernel ran at, from its own
+        # per-CTA cycle-counter and global-timer stamps
+        try:
+            kernel_clock = sa.sa_debug_kernel_clock()
+        except sa.SaError:
+            kernel_clock = None
         barrier()
         ms_local = start.elapsed_time(stop)
         attend_ms = [e[0][k].elapsed_time(e[1][k]) for e in evs for k in range(attends_per_chunk)]
@@ -763,15 +769,23 @@ def run_ours(args, w):
     peak_kind = (f"bf16 {'sustained' if long_region else 'burst'} ({peak_src}); timed region "
                  f"{region_s:.3f} s")
     per_clock = None
-    if clock_info and clock_info.get("sm_mhz"):
-        sms = torch.cuda.get_device_properties(dev).multi_processor_count
-        mhz = clock_info["sm_mhz"]
-        per_clock = {
-            "sm_mhz_median": mhz, "sms": sms,
-            "ms_x_mhz": attend_avg * mhz,
-            "flop_per_sm_clock": flops_rank / (attend_avg * 1e-3 * mhz * 1e6 * sms),
-            "dense_mma_flop_per_sm_clock": 8192,
-        }
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    if kernel_clock is not None or (clock_info and clock_info.get("sm_mhz")):
+        per_clock = {"sms": sms, "dense_mma_flop_per_sm_clock": 8192}
+        if kernel_clock is not None:
+            # The last timed attention launch by its own per-CTA stamps: the SM
+            # clock it ran at (cycle counter / global timer) and first start to
+            # last end. NVML can read the maximum clock while the SMs run slower.
+            mhz, span_us = kernel_clock
+            per_clock["kernel_last_launch"] = {
+                "sm_mhz": mhz, "span_ms": span_us * 1e-3,
+                "flop_per_sm_clock": flops_rank / (span_us * 1e-6 * mhz * 1e6 * sms)}
+        if clock_info and clock_info.get("sm_mhz"):
+            nv = clock_info["sm_mhz"]
+            per_clock["nvml_sm_mhz_median"] = nv
+            per_clock["ms_x_nvml_mhz"] = attend_avg * nv
+            per_clock["flop_per_sm_clock_at_nvml_mhz"] = flops_rank / (attend_avg * 1e-3 * nv * 1e6
+                                                                       * sms)
     append_bytes = appends_per_chunk * 2 * 2 * (w.batch * w.chunk_len * w.heads * w.head_dim * 2)
     # (per append of one tier: K and V, each read once and written once)
     append_gbs = append_bytes / (statistics.fmean(append_ms) * 1e-3) / 1e9

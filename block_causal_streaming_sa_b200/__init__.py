@@ -15,7 +15,7 @@ from ._binding import (  # noqa: F401
     sa_stage_keys,
     sa_stage_keys_frames, sa_attend_staged, sa_debug_attend_simt, sa_attend_noalloc, sa_debug_exp2,
     sa_debug_attend_stalled, sa_attend_sparse, sa_block_grid,
-    sa_chunk_count, sa_debug_inject_cuda_error, sa_debug_layout, sa_plan, sa_stream_plan, sa_slot_of,
+    sa_chunk_count, sa_debug_inject_cuda_error, sa_debug_kernel_clock, sa_debug_layout, sa_plan, sa_stream_plan, sa_slot_of,
     sa_get_status, last_error, SA_PAYLOAD_FP8, SA_PAYLOAD_BF16, sa_exchange_block_bytes,
     sa_exchange_pack, sa_exchange_unpack, sa_exchange_pack_to, sa_ipc_handle, sa_ipc_open,
     sa_ipc_close, sa_ipc_alloc, sa_ipc_free,

@@ -86,6 +86,7 @@ _SIGNATURES = {
     "sa_debug_attend_stalled": (_I, [_P, _P, _P, _P, _I, _P, _P]),
     "sa_chunk_count": (_I, [_P, _I]),
     "sa_debug_inject_cuda_error": (_I, [_P]),
+    "sa_debug_kernel_clock": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
     "sa_debug_layout": (_I, [_P, _I, _I32P, _I32P, _I]),
     "sa_plan": (_I, [_CFGP, ctypes.c_int32, _I32P, _I32P, _I32P, _I]),
     "sa_stream_plan": (_I, [_P, _I, _I, _I32P, _I32P, _I32P, _I]),
@@ -253,6 +254,15 @@ def sa_debug_inject_cuda_error(handle):
 
 def sa_chunk_count(handle, tier):
     return lib().sa_chunk_count(handle, tier)
+
+
+def sa_debug_kernel_clock():
+    """(SM MHz, span in us) of the most recent attention kernel on the current
+    device: the median over its CTAs of SM cycles per global-timer nanosecond,
+    and first CTA start to last CTA end. Synchronizes the device."""
+    mhz, span = ctypes.c_double(), ctypes.c_double()
+    _check(lib().sa_debug_kernel_clock(ctypes.byref(mhz), ctypes.byref(span)))
+    return mhz.value, span.value
 
 
 def sa_debug_layout(handle, tier, n):

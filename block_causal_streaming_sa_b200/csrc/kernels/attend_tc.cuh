@@ -258,6 +258,12 @@ __global__ void __launch_bounds__(384, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // clock record: global timer and SM cycles at the CTA's start and end (the
+  // condition re-read at the end rather than kept live through the kernel)
+  if (threadIdx.x == 0 && p.clock_stamps != nullptr && blockIdx.x < kMaxClockCtas) {
+    p.clock_stamps[4 * blockIdx.x] = ptx::globaltimer();
+    p.clock_stamps[4 * blockIdx.x + 1] = static_cast<unsigned long long>(clock64());
+  }
   const int n_qt = (p.L + T::BM - 1) / T::BM;
   const int n_pairs = (n_qt + 1) / 2;
   const int n_work = p.B * p.H * n_pairs;
@@ -911,6 +917,10 @@ __global__ void __launch_bounds__(384, 1)
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
+  if (threadIdx.x == 0 && p.clock_stamps != nullptr && blockIdx.x < kMaxClockCtas) {
+    p.clock_stamps[4 * blockIdx.x + 2] = ptx::globaltimer();
+    p.clock_stamps[4 * blockIdx.x + 3] = static_cast<unsigned long long>(clock64());
+  }
   if (warp == 1) ptx::tmem_dealloc(tmem, T::kTmemCols);
 }
 

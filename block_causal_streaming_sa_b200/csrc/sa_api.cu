@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <cstring>
 #include <initializer_list>
+#include <atomic>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -504,6 +505,9 @@ int max_groups(const sa_handle* h, bool source) {
   return h->d.S + h->d.W + (h->d.RF > 0 ? 1 : 0) + (source ? 1 : 0);
 }
 
+unsigned long long* clock_record(const sa_handle* h);
+void note_clock_grid(const sa_handle* h, unsigned grid);
+
 // Everything of AttendParams but the key source of the current chunk.
 void fill_common(sa_handle* h, int tier, int n_frames, bool source, const void* Q,
                  const void* Vc, void* O, float* lse, AttendParams* ap) {
@@ -532,6 +536,7 @@ void fill_common(sa_handle* h, int tier, int n_frames, bool source, const void* 
   ap->cache_elems = 2ULL * (d.S + d.R) * d.chunk_elems;
   ap->kcur_elems = 2ULL * d.chunk_elems;
   ap->ref_elems = 2ULL * d.ref_elems;
+  ap->clock_stamps = clock_record(h);
 }
 
 int check_attend_ptrs(sa_handle* h, const void* Q, const void* Vc, const void* O,
@@ -650,7 +655,9 @@ int attend_staged(sa_handle* h, const void* Q, const void* Vc, int step_is_final
     const int mode = block_mask != nullptr ? sa::kModeSparse
                      : aligned             ? sa::kModeAligned
                                            : sa::kModeDense;
-    launch_attend_tc(d.D, mode, attend_grid(d, ap.L, h->sm_count, ap.split_ok != 0), s, maps,
+    const unsigned grid = attend_grid(d, ap.L, h->sm_count, ap.split_ok != 0);
+    note_clock_grid(h, grid);
+    launch_attend_tc(d.D, mode, grid, s, maps,
                      ap);
   }
   cudaError_t e = cudaGetLastError();
@@ -748,25 +755,51 @@ bool current_ctx_id(unsigned long long* id) {
   return get_id(ctx, id) == CUDA_SUCCESS;
 }
 
-int noalloc_scratch(sa_handle* h, void** out) {
-  if (h->device < 0 || h->device >= kMaxDevices)
-    return h->fail(SA_ERR_UNSUPPORTED, "device ordinal too large for sa_attend_noalloc");
+// Device address of a static device array on `device` (current), from `table`
+// or looked up and cached there; an empty string on success, else the reason.
+std::string symbol_address(int device, const void* symbol, NoallocAddr* table, void** out) {
   unsigned long long ctx = 0;
-  if (!current_ctx_id(&ctx))
-    return h->fail(SA_ERR_CUDA, "sa_attend_noalloc: no current CUDA context");
+  if (!current_ctx_id(&ctx)) return "no current CUDA context";
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  NoallocAddr& a = g_noalloc_addr[h->device];
+  NoallocAddr& a = table[device];
   if (a.ptr == nullptr || a.ctx_id != ctx) {
     void* ptr = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_keys);
+    cudaError_t e = cudaGetSymbolAddress(&ptr, symbol);
     if (e != cudaSuccess || ptr == nullptr)
-      return h->fail(SA_ERR_CUDA, std::string("cudaGetSymbolAddress of the static key scratch: ") +
-                                      cudaGetErrorString(e));
+      return std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e);
     a.ptr = ptr;
     a.ctx_id = ctx;
   }
   *out = a.ptr;
+  return std::string();
+}
+
+int noalloc_scratch(sa_handle* h, void** out) {
+  if (h->device < 0 || h->device >= kMaxDevices)
+    return h->fail(SA_ERR_UNSUPPORTED, "device ordinal too large for sa_attend_noalloc");
+  const std::string why = symbol_address(h->device, g_noalloc_keys, g_noalloc_addr, out);
+  if (!why.empty()) return h->fail(SA_ERR_CUDA, "sa_attend_noalloc key scratch: " + why);
   return SA_OK;
+}
+
+// Clock record of the attention kernel (sa_debug_kernel_clock): per CTA the
+// global timer and the SM cycle counter at its start and end, for the most recent
+// attention launch on each device, and that launch's CTA count.
+static __device__ unsigned long long g_clock_stamps[sa::kMaxClockCtas * 4];
+NoallocAddr g_clock_addr[kMaxDevices] = {};
+std::atomic<int> g_clock_grid[kMaxDevices];
+
+// The record's device address, or null (the attention runs without it).
+unsigned long long* clock_record(const sa_handle* h) {
+  if (h->device < 0 || h->device >= kMaxDevices) return nullptr;
+  void* p = nullptr;
+  if (!symbol_address(h->device, g_clock_stamps, g_clock_addr, &p).empty()) return nullptr;
+  return static_cast<unsigned long long*>(p);
+}
+
+void note_clock_grid(const sa_handle* h, unsigned grid) {
+  if (h->device >= 0 && h->device < kMaxDevices)
+    g_clock_grid[h->device].store(static_cast<int>(grid));
 }
 
 int attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc, int step_is_final,
@@ -811,7 +844,9 @@ int attend_noalloc(sa_handle* h, const void* Q, const void* Kc, const void* Vc, 
   if (rc != SA_OK) return rc;
   AttendMaps maps{h->has_cache ? &h->tm_tier[tier] : &tm_keys, &tm_keys, &tm_v,
                   d.RF > 0 ? &h->tm_ref : &tm_keys, &tm_v, &tm_q};
-  launch_attend_tc(d.D, sa::kModeDense, attend_grid(d, d.L, h->sm_count, false), s, maps, ap);
+  const unsigned grid = attend_grid(d, d.L, h->sm_count, false);
+  note_clock_grid(h, grid);
+  launch_attend_tc(d.D, sa::kModeDense, grid, s, maps, ap);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
     return h->fail(SA_ERR_CUDA, std::string("attend launch: ") + cudaGetErrorString(e));
@@ -1344,6 +1379,49 @@ SA_API int sa_debug_exp2(int use_polynomial, const float* x, float* y, int n, sa
     g_error = std::string("exp2 probe launch: ") + cudaGetErrorString(e);
     return SA_ERR_CUDA;
   }
+  return SA_OK;
+}
+
+SA_API int sa_debug_kernel_clock(double* sm_mhz, double* span_us) {
+  if (sm_mhz == nullptr || span_us == nullptr) {
+    g_error = "sa_debug_kernel_clock: NULL output";
+    return SA_ERR_INVALID_ARG;
+  }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    g_error = "sa_debug_kernel_clock: no usable current device";
+    return SA_ERR_CUDA;
+  }
+  const int n = g_clock_grid[dev].load();
+  if (n <= 0) {
+    g_error = "sa_debug_kernel_clock: no attention has run on this device";
+    return SA_ERR_STATE;
+  }
+  const int ctas = n < sa::kMaxClockCtas ? n : sa::kMaxClockCtas;
+  std::vector<unsigned long long> st(4 * static_cast<size_t>(ctas));
+  if (cudaDeviceSynchronize() != cudaSuccess ||
+      cudaMemcpyFromSymbol(st.data(), g_clock_stamps, st.size() * sizeof(st[0])) != cudaSuccess) {
+    g_error = std::string("sa_debug_kernel_clock: ") + cudaGetErrorString(cudaGetLastError());
+    return SA_ERR_CUDA;
+  }
+  std::vector<double> mhz;
+  unsigned long long t0 = ~0ull, t1 = 0;
+  for (int c = 0; c < ctas; ++c) {
+    const unsigned long long* r = &st[4 * static_cast<size_t>(c)];
+    if (r[2] <= r[0] || r[3] <= r[1]) continue;  // not stamped by this launch
+    mhz.push_back(1e3 * static_cast<double>(r[3] - r[1]) / static_cast<double>(r[2] - r[0]));
+    t0 = std::min(t0, r[0]);
+    t1 = std::max(t1, r[2]);
+  }
+  if (mhz.empty()) {
+    g_error = "sa_debug_kernel_clock: the last launch left no stamps";
+    return SA_ERR_STATE;
+  }
+  std::sort(mhz.begin(), mhz.end());
+  const size_t k = mhz.size();
+  *sm_mhz = k % 2 ? mhz[k / 2] : 0.5 * (mhz[k / 2 - 1] + mhz[k / 2]);
+  *span_us = 1e-3 * static_cast<double>(t1 - t0);
   return SA_OK;
 }
 

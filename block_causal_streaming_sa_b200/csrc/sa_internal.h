@@ -123,6 +123,11 @@ struct AttendParams {
   unsigned long long cache_elems, kcur_elems, ref_elems;
   int debug_stall_producer;  // test hook: 1 = the TMA producer issues nothing, so the
                              // MMA warp's bounded wait runs out (timeout path)
+  // Clock record: per CTA (blockIdx.x < kMaxClockCtas) the global timer (ns) and
+  // the SM cycle counter at its start and at its end, or null.
+  unsigned long long* clock_stamps;  // [CTA][4]
 };
+
+constexpr int kMaxClockCtas = 1024;
 
 }  // namespace sa

@@ -304,6 +304,18 @@ SA_API int sa_debug_attend_stalled(sa_handle* h, const void* Q, const void* Kc, 
  * hook for the kernel's arithmetic; asynchronous on `stream`. */
 SA_API int sa_debug_exp2(int use_polynomial, const float* x, float* y, int n, sa_stream stream);
 
+/* Clock record of the most recent attention kernel (tensor-core path) that ran
+ * on the calling thread's current device, from any handle: every CTA stamps
+ * the global timer and its SM cycle counter when it starts and when it ends.
+ * *sm_mhz = the median over the CTAs of (SM cycles / timer ns) * 1000, the
+ * clock the kernel's SMs actually ran at (the clock a management library
+ * reports can stay at its maximum while the SMs run slower under power
+ * management); *span_us = first CTA start to last CTA end. Synchronizes the
+ * device first. SA_ERR_STATE when no attention has run on this device in this
+ * process; SA_ERR_CUDA without a usable device. Launches on several streams
+ * overwrite one record. */
+SA_API int sa_debug_kernel_clock(double* sm_mhz, double* span_us);
+
 /* Test hook for the host error path: the next call of this handle that would
  * launch device work fails with SA_ERR_CUDA before launching anything (as a
  * failed CUDA call would), leaving the handle's state unchanged; later calls

@@ -93,6 +93,14 @@ def test_create_without_gpu_fails_cleanly():
         sa.sa_create(_cfg(), 0x100000, 16)
 
 
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_kernel_clock_without_gpu_fails_cleanly():
+    mhz, span = ctypes.c_double(), ctypes.c_double()
+    rc = sa.lib().sa_debug_kernel_clock(ctypes.byref(mhz), ctypes.byref(span))
+    assert rc in (sa.SA_ERR_CUDA, sa.SA_ERR_STATE)
+    assert sa.lib().sa_debug_kernel_clock(None, None) == sa.SA_ERR_INVALID_ARG
+
+
 def test_null_handle_calls_fail_cleanly():
     lib = sa.lib()
     assert lib.sa_attend(None, None, None, None, 0, None, None, None) == sa.SA_ERR_INVALID_ARG

@@ -224,3 +224,23 @@ def test_fp16_range_of_rotated_pairs_is_flagged():
     h.append(CLEAN, Kn, Vn)
     h.attend(Q, Kc, Vc, True)
     assert h.status() == sa.SA_OK
+
+
+def test_kernel_clock_record_of_the_last_attention():
+    """sa_debug_kernel_clock reads the per-CTA stamps of the most recent attention
+    launch: a clock between 300 MHz and the part's 2.1 GHz ceiling, and a span
+    no longer than the launch as CUDA events time it."""
+    h = sa.StreamingAttention(W.config_dict())
+    Kn, Vn = W.tensor("Kn", 0).cuda(), W.tensor("Vn", 0).cuda()
+    h.append(NOISY, Kn, Vn)
+    h.append(CLEAN, Kn, Vn)
+    Q, Kc, Vc = _tensors(1)
+    h.attend(Q, Kc, Vc, False)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    h.attend(Q, Kc, Vc, True)
+    e1.record()
+    mhz, span_us = sa.sa_debug_kernel_clock()
+    assert 300.0 < mhz < 2100.0, mhz
+    assert 0.0 < span_us <= 1e3 * e0.elapsed_time(e1) + 5.0, (span_us, e0.elapsed_time(e1))
+    assert h.status() == sa.SA_OK
