@@ -31,7 +31,7 @@ __device__ __forceinline__ float2 rope_cs(const RopeTables& rt, int pair, int po
   pair -= rt.dt2;
   if (pair < rt.dh2) return __ldg(&rt.h[y * rt.dh2 + pair]);
   pair -= rt.dh2;
-  return __ldg(&rt.w[x * rt.dw2 + pair]);
+  return __ldg(&rt.w[pair * rt.tok_w + x]);
 }
 
 // Turn one bf16 pair by (cos, sin) in fp32; the result is rounded once to fp16,

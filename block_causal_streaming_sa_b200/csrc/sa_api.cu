@@ -1167,18 +1167,22 @@ SA_API int sa_create(const sa_config* cfg, void* dev_buf, size_t bytes, sa_handl
   const int n_tpos = d.RF + (d.S + d.W) * d.F;
   std::vector<float2> t(static_cast<size_t>(n_tpos) * d.dt2);
   std::vector<float2> th(static_cast<size_t>(d.th) * d.dh2), tw(static_cast<size_t>(d.tw) * d.dw2);
-  auto fill = [&](std::vector<float2>& tab, int npos, int npair) {
+  // t and h position-major ([pos][pair]); w pair-major ([pair][x]), so that the
+  // 32 rows of a warp, which lie at consecutive columns, read one pair's entries
+  // from consecutive addresses.
+  auto fill = [&](std::vector<float2>& tab, int npos, int npair, bool pair_major) {
     const double band = 2.0 * npair;
     for (int pos = 0; pos < npos; ++pos)
       for (int i = 0; i < npair; ++i) {
         const double a = pos * std::pow(static_cast<double>(d.theta), -2.0 * i / band);
-        tab[static_cast<size_t>(pos) * npair + i] =
-            make_float2(static_cast<float>(std::cos(a)), static_cast<float>(std::sin(a)));
+        const size_t at = pair_major ? static_cast<size_t>(i) * npos + pos
+                                     : static_cast<size_t>(pos) * npair + i;
+        tab[at] = make_float2(static_cast<float>(std::cos(a)), static_cast<float>(std::sin(a)));
       }
   };
-  fill(t, n_tpos, d.dt2);
-  fill(th, d.th, d.dh2);
-  fill(tw, d.tw, d.dw2);
+  fill(t, n_tpos, d.dt2, false);
+  fill(th, d.th, d.dh2, false);
+  fill(tw, d.tw, d.dw2, true);
   bool ok = cudaMemset(h->buf + d.off_status, 0, 1024) == cudaSuccess &&
             cudaMemset(h->buf + d.off_split_sem, 0, d.split_sem_bytes) == cudaSuccess;
   ok = ok && cudaMemcpy(h->buf + d.off_rope_t, t.data(), t.size() * sizeof(float2),

@@ -51,7 +51,7 @@ __device__ __forceinline__ bool in_bounds(unsigned* status, unsigned long long e
 struct RopeTables {
   const float2* t;  // [ref_frames + (S + W) * F][dt2]
   const float2* h;  // [tok_h][dh2]
-  const float2* w;  // [tok_w][dw2]
+  const float2* w;  // [dw2][tok_w] (pair-major: a warp's rows are consecutive columns)
   int dt2, dh2, dw2;
   int tok_h, tok_w, frame_tokens;  // frame_tokens = tok_h * tok_w
 };
