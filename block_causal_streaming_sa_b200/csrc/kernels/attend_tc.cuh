@@ -183,7 +183,12 @@ __device__ __noinline__ void epilogue(const AttendParams& p, uint32_t tO, bool a
   const size_t prow = ((static_cast<size_t>(slot) * 2 + i) * 2 + half) * T::BM + r;
   const size_t qrow = ((static_cast<size_t>(slot) * 2 + i) * 2 + (1 - half)) * T::BM + r;
   if (!SA_IN_BOUNDS(p.status, (prow > qrow ? prow : qrow) + 1, p.split_rows)) return;
-  float* po = p.split_o + prow * D;
+  // A half's partial rows are stored [D / 4][128 rows][4]: for one group of four
+  // columns a warp's 16-byte accesses cover 512 contiguous bytes (row-major rows,
+  // 512 bytes apart, made every warp access touch 32 lines; the merge's reads of
+  // them took ~29 K clocks at the end of the kernel's last round).
+  float4* pb = reinterpret_cast<float4*>(p.split_o + (prow - r) * D);
+  const float4* qb = reinterpret_cast<const float4*>(p.split_o + (qrow - r) * D);
 #pragma unroll 1
   for (int j = 0; j < D / 32; ++j) {
     uint32_t o[32];
@@ -193,7 +198,7 @@ __device__ __noinline__ void epilogue(const AttendParams& p, uint32_t tO, bool a
     }
 #pragma unroll
     for (int c = 0; c < 32; c += 4)
-      reinterpret_cast<float4*>(po + j * 32)[c / 4] =
+      pb[((j * 32 + c) / 4) * T::BM + r] =
           seen ? make_float4(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv,
                              __uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv)
                : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -206,8 +211,8 @@ __device__ __noinline__ void epilogue(const AttendParams& p, uint32_t tO, bool a
   const float lse_other = __ldcg(p.split_lse + qrow);
   const float l0 = half == 0 ? lse_own : lse_other;
   const float l1 = half == 0 ? lse_other : lse_own;
-  const float* o0 = half == 0 ? po : p.split_o + qrow * D;
-  const float* o1 = half == 0 ? p.split_o + qrow * D : po;
+  const float4* o0 = half == 0 ? pb : qb;  // half 0's block, then half 1's
+  const float4* o1 = half == 0 ? qb : pb;
   const float mx2 = fmaxf(l0, l1);
   float w0 = 0.f, w1 = 0.f, lse_tot = -INFINITY;
   if (mx2 != -INFINITY) {
@@ -217,18 +222,27 @@ __device__ __noinline__ void epilogue(const AttendParams& p, uint32_t tO, bool a
     w1 = e1 / (e0 + e1);
   }
   if (valid) {
+    // 32 columns of both partial rows requested at a time (this merge ends the
+    // kernel's last round)
 #pragma unroll 1
-    for (int c = 0; c < D; c += 8) {
-      const float4 a0 = __ldcg(reinterpret_cast<const float4*>(o0 + c));
-      const float4 a1 = __ldcg(reinterpret_cast<const float4*>(o0 + c + 4));
-      const float4 b0 = __ldcg(reinterpret_cast<const float4*>(o1 + c));
-      const float4 b1 = __ldcg(reinterpret_cast<const float4*>(o1 + c + 4));
-      uint4 q4;
-      q4.x = ptx::pack_bf16x2(fmaf(w1, b0.x, w0 * a0.x), fmaf(w1, b0.y, w0 * a0.y));
-      q4.y = ptx::pack_bf16x2(fmaf(w1, b0.z, w0 * a0.z), fmaf(w1, b0.w, w0 * a0.w));
-      q4.z = ptx::pack_bf16x2(fmaf(w1, b1.x, w0 * a1.x), fmaf(w1, b1.y, w0 * a1.y));
-      q4.w = ptx::pack_bf16x2(fmaf(w1, b1.z, w0 * a1.z), fmaf(w1, b1.w, w0 * a1.w));
-      st_v4(dst + c / 8, q4);
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      float4 a[8], bv[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        a[k] = __ldcg(o0 + (c0 / 4 + k) * T::BM + r);
+        bv[k] = __ldcg(o1 + (c0 / 4 + k) * T::BM + r);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; k += 2) {
+        uint4 q4;
+        q4.x = ptx::pack_bf16x2(fmaf(w1, bv[k].x, w0 * a[k].x), fmaf(w1, bv[k].y, w0 * a[k].y));
+        q4.y = ptx::pack_bf16x2(fmaf(w1, bv[k].z, w0 * a[k].z), fmaf(w1, bv[k].w, w0 * a[k].w));
+        q4.z = ptx::pack_bf16x2(fmaf(w1, bv[k + 1].x, w0 * a[k + 1].x),
+                                fmaf(w1, bv[k + 1].y, w0 * a[k + 1].y));
+        q4.w = ptx::pack_bf16x2(fmaf(w1, bv[k + 1].z, w0 * a[k + 1].z),
+                                fmaf(w1, bv[k + 1].w, w0 * a[k + 1].w));
+        st_v4(dst + (c0 + 4 * k) / 8, q4);
+      }
     }
     if (lse_ok) p.lse[lse_idx] = lse_tot;
   }

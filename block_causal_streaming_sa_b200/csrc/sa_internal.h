@@ -113,7 +113,7 @@ struct AttendParams {
   // its tiles are split into two key-range halves; each half writes a
   // normalised fp32 partial row and its lse, and per row the second finisher
   // (atomic counter) merges both. Regions sized for kMaxSplitSlots tiles.
-  float* split_o;    // [slot][query tile 0/1][half][128 rows][D]
+  float* split_o;    // [slot][query tile 0/1][half][D / 4][128 rows][4]
   float* split_lse;  // [slot][query tile][half][128 rows]
   int* split_sem;    // [slot][query tile][128 rows], zero between launches
   int split_ok;
