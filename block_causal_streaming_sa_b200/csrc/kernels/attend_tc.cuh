@@ -130,6 +130,46 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   return v;
 }
 
+// Store columns [col0, col0 + 32) of a warp's 32 O rows (bf16): lane l passes its
+// row's 16 packed words; they go through the warp's staging rows in shared
+// memory (stride kQRawRow bytes, the warp's own raw-query rows, unused once its
+// unit's last key tile is done) and come back so that each store instruction
+// writes whole 64-byte (D = 64: 32-byte) segments of 8 (16) rows. Row k of the
+// warp is stored when k < n_rows, at row_off0 + k * row_stride. (A thread
+// storing its own row in 16-byte pieces, rows H * D * 2 bytes apart, made every
+// store instruction touch 32 lines.)
+template <int D>
+__device__ __forceinline__ void warp_store_cols(const AttendParams& p, unsigned long long row_off0,
+                                                unsigned long long row_stride, int n_rows,
+                                                const uint32_t (&w)[16], uint32_t stage, int lane,
+                                                int col0) {
+  using T = TcShape<D>;
+  constexpr int PW = T::kQRawRow >= 64 ? 64 : 32;  // staged bytes per row and pass
+  constexpr int PP = PW / 16;                       // 16-byte pieces per row and pass
+  constexpr int RPI = 32 / PP;                      // rows per store instruction
+#pragma unroll
+  for (int pass = 0; pass < 64 / PW; ++pass) {
+    __syncwarp();  // the previous pass has read the staging rows
+#pragma unroll
+    for (int q = 0; q < PP; ++q) {
+      const int wi = (pass * PP + q) * 4;
+      st_shared_v4(stage + lane * T::kQRawRow + q * 16,
+                   make_uint4(w[wi], w[wi + 1], w[wi + 2], w[wi + 3]));
+    }
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < PP; ++k) {
+      const int row = k * RPI + lane / PP, piece = lane % PP;
+      const uint4 v = ld_shared_v4(stage + row * T::kQRawRow + piece * 16);
+      const unsigned long long off =
+          row_off0 + row * row_stride + col0 + pass * (PW / 2) + piece * 8;
+      if (row < n_rows && SA_IN_BOUNDS(p.status, off + 8, p.q_elems))
+        st_v4(p.o + off, v);
+    }
+  }
+  __syncwarp();
+}
+
 // Epilogue of one query row of a work unit; a function of its own so that its
 // registers do not count against the score loop's (it runs once per unit).
 // O / l -> bf16 row of [B, L, H, D] and the natural-log LSE; a row that saw no
@@ -152,6 +192,16 @@ __device__ __noinline__ void epilogue(const AttendParams& p, uint32_t tO, bool a
                       SA_IN_BOUNDS(p.status, static_cast<unsigned long long>(lse_idx) + 1,
                                    p.lse_elems);
   if (half < 0) {
+    // the warp's rows are consecutive tokens; the valid ones a prefix of its lanes.
+    // Staging: the warp's raw-query rows of this tile (the dynamic shared memory
+    // base is re-derived here, as the kernel aligns it, rather than passed in).
+    const int lane = r & 31;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = ptx::smem_addr(smem_raw);
+    const uint32_t stage = raw_addr + ((1024u - (raw_addr & 1023u)) & 1023u) + T::kOffQRaw +
+                           static_cast<uint32_t>((i * T::BM + (r & ~31)) * T::kQRawRow);
+    const int n_rows = __popc(__ballot_sync(0xffffffffu, valid));
+    const unsigned long long row_off0 = __shfl_sync(0xffffffffu, row_off, 0);
 #pragma unroll 1
     for (int j = 0; j < D / 32; ++j) {
       uint32_t o[32];
@@ -159,23 +209,14 @@ __device__ __noinline__ void epilogue(const AttendParams& p, uint32_t tO, bool a
         ptx::tmem_ld32(tO + j * 32, o);
         ptx::tmem_wait_ld();
       }
-      if (valid) {
+      uint32_t wv[16];
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          uint4 q4 = make_uint4(0u, 0u, 0u, 0u);
-          if (seen) {
-            q4.x = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv,
-                                    __uint_as_float(o[8 * v + 1]) * inv);
-            q4.y = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv,
-                                    __uint_as_float(o[8 * v + 3]) * inv);
-            q4.z = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv,
-                                    __uint_as_float(o[8 * v + 5]) * inv);
-            q4.w = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv,
-                                    __uint_as_float(o[8 * v + 7]) * inv);
-          }
-          st_v4(dst + j * 4 + v, q4);
-        }
-      }
+      for (int k = 0; k < 16; ++k)
+        wv[k] = seen ? ptx::pack_bf16x2(__uint_as_float(o[2 * k]) * inv,
+                                        __uint_as_float(o[2 * k + 1]) * inv)
+                     : 0u;
+      warp_store_cols<D>(p, row_off0, static_cast<unsigned long long>(p.H) * D, n_rows, wv,
+                         stage, lane, j * 32);
     }
     if (valid && lse_ok) p.lse[lse_idx] = lse_own;
     return;
