@@ -185,23 +185,24 @@ __device__ __noinline__ void epilogue(const AttendParams& p, uint32_t tO, bool a
   const bool seen = lsum > 0.f;
   const float inv = seen ? 1.f / lsum : 0.f;
   const float lse_own = seen ? (m + __log2f(lsum)) * 0.69314718055994531f : -INFINITY;
-  uint4* dst = reinterpret_cast<uint4*>(p.o + row_off);
   // checked build: the row of O and the lse entry lie inside their buffers
   valid = valid && SA_IN_BOUNDS(p.status, row_off + D, p.q_elems);
   const bool lse_ok = valid && p.lse != nullptr &&
                       SA_IN_BOUNDS(p.status, static_cast<unsigned long long>(lse_idx) + 1,
                                    p.lse_elems);
+  // The warp's rows are consecutive tokens and its valid rows a prefix of its
+  // lanes; O goes out through the warp's staging rows (its raw-query rows of this
+  // tile; the dynamic shared memory base is re-derived here as the kernel aligns
+  // it, rather than passed in).
+  const int lane = r & 31;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = ptx::smem_addr(smem_raw);
+  const uint32_t stage = raw_addr + ((1024u - (raw_addr & 1023u)) & 1023u) + T::kOffQRaw +
+                         static_cast<uint32_t>((i * T::BM + (r & ~31)) * T::kQRawRow);
+  const int n_rows = __popc(__ballot_sync(0xffffffffu, valid));
+  const unsigned long long row_off0 = __shfl_sync(0xffffffffu, row_off, 0);
+  const unsigned long long row_stride = static_cast<unsigned long long>(p.H) * D;
   if (half < 0) {
-    // the warp's rows are consecutive tokens; the valid ones a prefix of its lanes.
-    // Staging: the warp's raw-query rows of this tile (the dynamic shared memory
-    // base is re-derived here, as the kernel aligns it, rather than passed in).
-    const int lane = r & 31;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw_addr = ptx::smem_addr(smem_raw);
-    const uint32_t stage = raw_addr + ((1024u - (raw_addr & 1023u)) & 1023u) + T::kOffQRaw +
-                           static_cast<uint32_t>((i * T::BM + (r & ~31)) * T::kQRawRow);
-    const int n_rows = __popc(__ballot_sync(0xffffffffu, valid));
-    const unsigned long long row_off0 = __shfl_sync(0xffffffffu, row_off, 0);
 #pragma unroll 1
     for (int j = 0; j < D / 32; ++j) {
       uint32_t o[32];
@@ -215,15 +216,16 @@ __device__ __noinline__ void epilogue(const AttendParams& p, uint32_t tO, bool a
         wv[k] = seen ? ptx::pack_bf16x2(__uint_as_float(o[2 * k]) * inv,
                                         __uint_as_float(o[2 * k + 1]) * inv)
                      : 0u;
-      warp_store_cols<D>(p, row_off0, static_cast<unsigned long long>(p.H) * D, n_rows, wv,
-                         stage, lane, j * 32);
+      warp_store_cols<D>(p, row_off0, row_stride, n_rows, wv, stage, lane, j * 32);
     }
     if (valid && lse_ok) p.lse[lse_idx] = lse_own;
     return;
   }
   const size_t prow = ((static_cast<size_t>(slot) * 2 + i) * 2 + half) * T::BM + r;
   const size_t qrow = ((static_cast<size_t>(slot) * 2 + i) * 2 + (1 - half)) * T::BM + r;
-  if (!SA_IN_BOUNDS(p.status, (prow > qrow ? prow : qrow) + 1, p.split_rows)) return;
+  if (!__all_sync(0xffffffffu,
+                  SA_IN_BOUNDS(p.status, (prow > qrow ? prow : qrow) + 1, p.split_rows)))
+    return;
   // A half's partial rows are stored [D / 4][128 rows][4]: for one group of four
   // columns a warp's 16-byte accesses cover 512 contiguous bytes (row-major rows,
   // 512 bytes apart, made every warp access touch 32 lines; the merge's reads of
@@ -245,9 +247,15 @@ __device__ __noinline__ void epilogue(const AttendParams& p, uint32_t tO, bool a
                : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   p.split_lse[prow] = lse_own;
+  // One counter per warp of rows: the warp that finds the other half's warp done
+  // merges all 32 rows, so the merge's stores can go through the staging rows as
+  // well. Every lane's partial row is performed before its warp counts.
   __threadfence();
-  int* sem = p.split_sem + (static_cast<size_t>(slot) * 2 + i) * T::BM + r;
-  if (atomicAdd(sem, 1) != 1) return;  // the other half merges
+  __syncwarp();
+  int* sem = p.split_sem + (static_cast<size_t>(slot) * 2 + i) * T::BM + (r & ~31);
+  int prev = 0;
+  if (lane == 0) prev = atomicAdd(sem, 1);
+  if (__shfl_sync(0xffffffffu, prev, 0) != 1) return;  // the other half's warp merges
   __threadfence();
   const float lse_other = __ldcg(p.split_lse + qrow);
   const float l0 = half == 0 ? lse_own : lse_other;
@@ -262,32 +270,28 @@ __device__ __noinline__ void epilogue(const AttendParams& p, uint32_t tO, bool a
     w0 = e0 / (e0 + e1);
     w1 = e1 / (e0 + e1);
   }
-  if (valid) {
-    // 32 columns of both partial rows requested at a time (this merge ends the
-    // kernel's last round)
+  // 32 columns of both partial rows requested at a time (this merge ends the
+  // kernel's last round)
 #pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      float4 a[8], bv[8];
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    float4 a[8], bv[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        a[k] = __ldcg(o0 + (c0 / 4 + k) * T::BM + r);
-        bv[k] = __ldcg(o1 + (c0 / 4 + k) * T::BM + r);
-      }
-#pragma unroll
-      for (int k = 0; k < 8; k += 2) {
-        uint4 q4;
-        q4.x = ptx::pack_bf16x2(fmaf(w1, bv[k].x, w0 * a[k].x), fmaf(w1, bv[k].y, w0 * a[k].y));
-        q4.y = ptx::pack_bf16x2(fmaf(w1, bv[k].z, w0 * a[k].z), fmaf(w1, bv[k].w, w0 * a[k].w));
-        q4.z = ptx::pack_bf16x2(fmaf(w1, bv[k + 1].x, w0 * a[k + 1].x),
-                                fmaf(w1, bv[k + 1].y, w0 * a[k + 1].y));
-        q4.w = ptx::pack_bf16x2(fmaf(w1, bv[k + 1].z, w0 * a[k + 1].z),
-                                fmaf(w1, bv[k + 1].w, w0 * a[k + 1].w));
-        st_v4(dst + (c0 + 4 * k) / 8, q4);
-      }
+    for (int k = 0; k < 8; ++k) {
+      a[k] = __ldcg(o0 + (c0 / 4 + k) * T::BM + r);
+      bv[k] = __ldcg(o1 + (c0 / 4 + k) * T::BM + r);
     }
-    if (lse_ok) p.lse[lse_idx] = lse_tot;
+    uint32_t wv[16];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      wv[2 * k] = ptx::pack_bf16x2(fmaf(w1, bv[k].x, w0 * a[k].x), fmaf(w1, bv[k].y, w0 * a[k].y));
+      wv[2 * k + 1] =
+          ptx::pack_bf16x2(fmaf(w1, bv[k].z, w0 * a[k].z), fmaf(w1, bv[k].w, w0 * a[k].w));
+    }
+    warp_store_cols<D>(p, row_off0, row_stride, n_rows, wv, stage, lane, c0);
   }
-  *sem = 0;  // ready for the next launch
+  if (valid && lse_ok) p.lse[lse_idx] = lse_tot;
+  __syncwarp();
+  if (lane == 0) *sem = 0;  // ready for the next launch
 }
 
 template <int D, int kMode>

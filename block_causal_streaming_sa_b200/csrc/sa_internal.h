@@ -115,7 +115,7 @@ struct AttendParams {
   // (atomic counter) merges both. Regions sized for kMaxSplitSlots tiles.
   float* split_o;    // [slot][query tile 0/1][half][D / 4][128 rows][4]
   float* split_lse;  // [slot][query tile][half][128 rows]
-  int* split_sem;    // [slot][query tile][128 rows], zero between launches
+  int* split_sem;    // [slot][query tile][128 rows]: entry 32 w counts warp w of the rows; zero between launches
   int split_ok;
   // Buffer sizes for the checked build's bounds checks (elements): Q and O, lse,
   // bit-row words, split-tail rows; for the SIMT kernel the key sources too.
