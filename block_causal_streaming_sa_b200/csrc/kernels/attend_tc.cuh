@@ -809,7 +809,16 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int cc = 0; cc < 8; ++cc)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) cs[cc][j] = rope_cs(p.rope, 4 * (c8 + cc) + j, td0 + f, y, x);
+            for (int j = 0; j < 4; ++j) {
+              // block-sparse units are short, so their start weighs: the band of
+              // each pair resolved at compile time there (in the dense and aligned
+              // instantiations it moved the score loop's register allocation and
+              // cost ~1 % per clock; sparse gained 2-2.5 %)
+              if constexpr (kSparse)
+                cs[cc][j] = rope_cs_d<D>(p.rope, 4 * (c8 + cc) + j, td0 + f, y, x);
+              else
+                cs[cc][j] = rope_cs(p.rope, 4 * (c8 + cc) + j, td0 + f, y, x);
+            }
 #pragma unroll
           for (int cc = 0; cc < 8; ++cc) {
             const int c = c8 + cc;

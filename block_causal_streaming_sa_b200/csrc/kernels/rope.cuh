@@ -34,6 +34,19 @@ __device__ __forceinline__ float2 rope_cs(const RopeTables& rt, int pair, int po
   return __ldg(&rt.w[pair * rt.tok_w + x]);
 }
 
+// The same with the band sizes of head dim D fixed at compile time (temporal
+// D - 4 (D/6) dims, row and column D/3 each, as the handle's tables are built):
+// with `pair` a constant after unrolling, each call is one load from a known
+// table, so a row's loads are all issued back to back.
+template <int D>
+__device__ __forceinline__ float2 rope_cs_d(const RopeTables& rt, int pair, int pos_t, int y,
+                                            int x) {
+  constexpr int dt2 = (D - 4 * (D / 6)) / 2, dh2 = D / 6;
+  if (pair < dt2) return __ldg(&rt.t[pos_t * dt2 + pair]);
+  if (pair < dt2 + dh2) return __ldg(&rt.h[y * dh2 + (pair - dt2)]);
+  return __ldg(&rt.w[(pair - dt2 - dh2) * rt.tok_w + x]);
+}
+
 // Turn one bf16 pair by (cos, sin) in fp32; the result is rounded once to fp16,
 // the operand type of the score MMA (11 significant bits instead of bf16's 8).
 __device__ __forceinline__ uint32_t rope_pair(uint32_t ab, float2 cs) {
