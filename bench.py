@@ -85,13 +85,25 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def kernel_code_hash(path):
+    """First 16 hex digits of the SHA-256 of a CUDA source with its // comments
+    and blank lines removed and each line stripped, so that an edit to comments
+    alone keeps the hash (and a profile taken on that code stays valid)."""
+    lines = []
+    for line in open(path, encoding="utf-8").read().splitlines():
+        code = re.sub(r"//.*$", "", line).strip()
+        if code:
+            lines.append(code)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()[:16]
+
+
 def kernel_traffic(kernel_file, workload):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the kernel source as it is now; else None."""
+    the kernel code as it is now (comments aside); else None."""
     src = os.path.join(ROOT, "block_causal_streaming_sa_b200", "csrc", "kernels", kernel_file)
     summ = os.path.join(ROOT, "profiles", f"attend_tc_{workload}.txt")
     try:
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        sha = kernel_code_hash(src)
         text = open(summ).read()
     except OSError:
         return None

@@ -23,15 +23,18 @@
 //    operands K-major in shared memory) into TMEM, then O_i += P_i V (TS form,
 //    bf16: P_i read from TMEM, written over the upper half of S_i, V MN-major
 //    in shared memory); the two query tiles ping-pong so one tile's softmax
-//    overlaps the other's MMAs;
+//    overlaps the other's MMAs. It also issues the TMA copy of each query tile
+//    of the next work unit as soon as this unit's O of that tile is final, so
+//    the copy runs under the epilogue;
 //  * warps 4-7 / 8-11: one warpgroup per query tile, thread = query row =
-//    TMEM lane. Each writes its rotated query tile into shared memory, runs the
+//    TMEM lane. Each turns its row of the query tile in shared memory, runs the
 //    online softmax on S rows read from TMEM in one round trip (no cross-thread
 //    reduction: a thread owns a whole row; max as an 8-way tree of 3-input
 //    maxima, scale-and-subtract and the row sum in packed fp32x2 instructions,
 //    1 exponential in 8 on the FMA pipe by a fitted polynomial), writes P
 //    back as bf16, rescales O in TMEM only when the running max grows by more
-//    than 2^8, and calls the epilogue;
+//    than 2^8, and calls the epilogue, which stores O through per-warp staging
+//    in shared memory (64-byte row segments per store instruction);
 //  * registers: launched at 168 per thread (384 threads), warpgroup 0 (warps
 //    0-3: producer, MMA issuer, two idle) gives registers back with setmaxnreg
 //    (104) and the softmax warpgroups take them (200), so a whole 128-score row
@@ -44,7 +47,7 @@
 //  * work units: rounds of gridDim.x work tiles; when the last round holds at
 //    most half a grid of tiles, each of them is split by attended chunks into
 //    two halves run by two CTAs, which write normalised fp32 partial rows and
-//    their log-sum-exp; per row, the second half to finish merges both;
+//    their log-sum-exp; per warp of rows, the second half to finish merges both;
 //  * block-sparse: the mask arrives as bit rows (one per query tile); step j of
 //    a work tile loads and multiplies the j-th flagged key tile of each of its
 //    two query tiles, so the ping-pong of the dense loop is kept (a key tile
